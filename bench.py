@@ -1,0 +1,548 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 paged KV-cache hot path.
+
+Headline workload (one "step"): the decode-batch-64 configuration — store_kvcache
+of the 64 new tokens through the slot mapping, then paged decode attention of the
+64 sequences (16 q heads / 8 kv heads, head dim 128, block size 256, contexts
+uniform in [512, 4096]) — with the whole pool resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). Under torchrun every rank runs its own batch of the
+same shape (independent sequences, no collective): weak scaling, value = all
+ranks' bytes / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, SENTINEL_BF16, generate  # noqa: E402
+
+METRIC = ("paged-attn decode achieved HBM GB/s (% of B200 peak); "
+          "decode steps/s at batch 64")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+DATASHEET_HBM_GBS = 8000.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------- utils
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), \
+            float(d.get("bf16_tflops_sustained", d.get("bf16_tflops", FALLBACK_BF16_TFLOPS))), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def file_hash(*paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+DECODE_SRC = ("paged_kv_cache_442_b200/csrc/decode.cu", "paged_kv_cache_442_b200/csrc/pa_ptx.cuh")
+PREFILL_SRC = ("paged_kv_cache_442_b200/csrc/prefill.cu", "paged_kv_cache_442_b200/csrc/pa_ptx.cuh")
+
+
+def recorded_traffic(name, srcs):
+    """Per-launch DRAM bytes from a committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", f"{name}.traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != file_hash(*srcs):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while a region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0=None, t1=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            if t0 is not None and not (t0 - 0.06 <= ts <= t1 + 0.06):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in timed region"],
+                    "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- byte/flop counts
+def decode_bytes(w):
+    """Algorithmic bytes of one decode: K/V rows of every visible position, q, out."""
+    kv = int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+    return kv + qo
+
+
+def store_bytes(w):
+    """new k/v read + written once each."""
+    return 2 * 2 * len(w.new_slots) * w.num_kv_heads * w.head_dim * 2
+
+
+def prefill_flops(w):
+    """Causal-exact: 4*D flops per (query, head, visible key)."""
+    tot = 0
+    for s in range(w.num_seqs):
+        n = int(w.new_lens[s])
+        ctx = int(w.context_lens[s])
+        first = ctx - n
+        # sum over i of (first + i + 1)
+        tot += n * (first + 1) + n * (n - 1) // 2
+    return 4 * w.head_dim * w.num_q_heads * tot
+
+
+def prefill_bytes(w):
+    kv = int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * int(w.new_lens.sum()) * w.num_q_heads * w.head_dim * 2
+    return kv + qo
+
+
+# --------------------------------------------------------------------------- GPU arm
+class GpuRunner:
+    def __init__(self, w, torch, pa, partition_size=0):
+        self.w, self.torch, self.pa = w, torch, pa
+        dev = torch.device("cuda")
+        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        fill = int(np.uint16(SENTINEL_BF16).view(np.int16))
+        self.k_cache = torch.full(shape, fill, dtype=torch.int16, device=dev).view(torch.bfloat16)
+        self.v_cache = torch.full(shape, fill, dtype=torch.int16, device=dev).view(torch.bfloat16)
+
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        def i32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+        if len(w.setup_slots):
+            # untimed setup: the cached context, written in chunks through the library
+            n = len(w.setup_slots)
+            step = 1 << 18
+            for s0 in range(0, n, step):
+                idx = np.arange(s0, min(n, s0 + step))
+                pa.pa_store_kvcache(bf(w.src_k[w.setup_src[idx]]), bf(w.src_v[w.setup_src[idx]]),
+                                    self.k_cache, self.v_cache, i32(w.setup_slots[idx]))
+        self.q = bf(w.q)
+        self.new_k = bf(w.new_k) if len(w.new_slots) else None
+        self.new_v = bf(w.new_v) if len(w.new_slots) else None
+        self.new_slots = i32(w.new_slots)
+        self.block_tables = i32(w.block_tables)
+        self.context_lens = i32(w.context_lens)
+        self.cu = i32(w.cu_seqlens_q)
+        self.out = torch.empty_like(self.q)
+        if w.kind == "decode":
+            self.ws, self.P = pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads,
+                                                  w.head_dim, w.max_context_len, partition_size)
+        self.max_q = int(np.max(np.diff(w.cu_seqlens_q))) if w.num_seqs else 0
+        torch.cuda.synchronize()
+
+    def store(self, k=None, v=None, slots=None):
+        if self.new_k is None and k is None:
+            return 0
+        self.pa.pa_store_kvcache(self.new_k if k is None else k, self.new_v if v is None else v,
+                                 self.k_cache, self.v_cache, self.new_slots if slots is None else slots)
+        return 1
+
+    def attend(self, q=None, ctx=None, bt=None, out=None):
+        w, pa = self.w, self.pa
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        ctx = self.context_lens if ctx is None else ctx
+        bt = self.block_tables if bt is None else bt
+        if w.kind == "decode":
+            pa.pa_decode(out, q, self.k_cache, self.v_cache, bt, ctx, w.scale,
+                         w.max_context_len, self.P, self.ws)
+            return 2 if self.ws is not None else 1
+        pa.pa_prefill(out, q, self.k_cache, self.v_cache, bt, self.cu, ctx, w.scale, self.max_q)
+        return 1
+
+    def step(self):
+        return self.store() + self.attend()
+
+
+def time_steps(runner, torch, steps, warmup, flush_buf, barrier=None):
+    """Per-step device time (ms) of `steps` steps, L2 flushed before each step.
+
+    Returns (total step ms, attention-call ms list, launches per step)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush_buf.add_(1)
+        runner.step()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    launches = 0
+    for i in range(steps):
+        flush_buf.add_(1)                       # write 256 MiB: evicts the previous step from L2
+        a, b, c = ev[i]
+        a.record(stream)
+        launches += runner.store()
+        b.record(stream)
+        launches += runner.attend()
+        c.record(stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    return sum(step_ms), attn_ms, launches // steps
+
+
+def time_e2e(runner, torch, steps, warmup):
+    """Same step through the host: pinned host inputs copied in, output copied out."""
+    w = runner.w
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_q = pin(runner.q)
+    h_k = pin(runner.new_k) if runner.new_k is not None else None
+    h_v = pin(runner.new_v) if runner.new_v is not None else None
+    h_slots = pin(runner.new_slots)
+    h_ctx = pin(runner.context_lens)
+    h_bt = pin(runner.block_tables)
+    h_out = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+    d_q, d_ctx, d_bt = torch.empty_like(runner.q), torch.empty_like(runner.context_lens), \
+        torch.empty_like(runner.block_tables)
+    d_k = torch.empty_like(runner.new_k) if h_k is not None else None
+    d_v = torch.empty_like(runner.new_v) if h_v is not None else None
+    d_slots = torch.empty_like(runner.new_slots)
+    d_out = torch.empty_like(runner.out)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_ctx, h_bt) if t is not None)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def one():
+        d_q.copy_(h_q, non_blocking=True)
+        d_ctx.copy_(h_ctx, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_slots.copy_(h_slots, non_blocking=True)
+        if d_k is not None:
+            d_k.copy_(h_k, non_blocking=True)
+            d_v.copy_(h_v, non_blocking=True)
+            runner.store(d_k, d_v, d_slots)
+        runner.attend(d_q, d_ctx, d_bt, d_out)
+        h_out.copy_(d_out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e), h2d, d2h
+
+
+# --------------------------------------------------------------------------- CPU (oracle) arm
+def oracle_pools_for(w):
+    """The oracle's own pools: setup rows and this step's new rows, stored by the oracle."""
+    import oracle
+    kc, vc = w.empty_pool(), w.empty_pool()
+    if len(w.setup_slots):
+        kc, vc = oracle.store_kvcache(kc, vc, w.setup_k, w.setup_v, w.setup_slots)
+    if len(w.new_slots):
+        kc, vc = oracle.store_kvcache(kc, vc, w.new_k, w.new_v, w.new_slots)
+    return kc, vc
+
+
+def oracle_decode_one(w, pools, s):
+    """Oracle decode of sequence s; returns (seconds, algorithmic bytes)."""
+    import oracle
+    kc, vc = pools
+    idx = np.array([s])
+    t0 = time.perf_counter()
+    oracle.decode(w.q[idx], kc, vc, w.block_tables[idx], w.context_lens[idx], w.scale)
+    dt = time.perf_counter() - t0
+    nbytes = int(w.context_lens[s]) * w.num_kv_heads * w.head_dim * 4 + 2 * w.num_q_heads * w.head_dim * 2
+    return dt, nbytes
+
+
+def host_threads():
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        blas = cores
+    return cores, blas
+
+
+def cpu_oracle_time(w, budget_s=12.0):
+    """The oracle (as it stands) decoding sequences one at a time for ~budget_s.
+
+    Returns (seconds, bytes, sequences decoded, cores, blas threads)."""
+    pools = oracle_pools_for(w)
+    tot_t, tot_b, n = 0.0, 0, 0
+    while tot_t < budget_s:
+        dt, nb = oracle_decode_one(w, pools, n % w.num_seqs)
+        tot_t += dt
+        tot_b += nb
+        n += 1
+    cores, blas = host_threads()
+    return tot_t, tot_b, n, cores, blas
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_b64")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the extra per-configuration measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--partition-size", type=int, default=0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args, cfg, world)
+        return
+
+    import torch
+    import paged_kv_cache_442_b200 as pa
+    torch.cuda.set_device(local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    hbm_peak, tf_peak, tf_sustained, peak_src = peaks()
+    # every rank decodes its own batch of the same shape (weak scaling)
+    w = generate(cfg) if rank == 0 else _rank_workload(cfg, rank)
+    runner = GpuRunner(w, torch, pa, args.partition_size)
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    t0 = time.time()
+    total_ms, attn_ms, launches_per_step = time_steps(runner, torch, args.steps, args.warmup, flush,
+                                                      barrier)
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+
+    step_ms = total_ms / args.steps
+    if pg is not None:
+        t = torch.tensor([step_ms], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        step_ms = float(t.item())
+    bytes_step = (decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)) + store_bytes(w)
+    value = world * bytes_step / (step_ms * 1e-3) / 1e9
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
+    achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
+    e2e_step_ms = e2e_ms / min(args.steps, 500)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "num_blocks": w.num_blocks,
+                   "context_lens": f"{cfg.ctx_dist}[{cfg.ctx_lo},{cfg.ctx_hi}] sum={int(w.context_lens.sum())}",
+                   "partition_size": getattr(runner, "P", None),
+                   "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed before every step (256 MiB write, outside the step events)"},
+        "steps_per_s": round(1e3 / step_ms * world, 1),
+        "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
+        "pct_of_datasheet_8tbs": round(100 * value / world / DATASHEET_HBM_GBS, 1),
+        "bytes_per_step": bytes_step,
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
+                     "algorithmic_bytes_per_launch": attn_bytes,
+                     "avg_launch_us": round(attn_avg_ms * 1e3, 2),
+                     "traffic": recorded_traffic(cfg.name + ".decode", DECODE_SRC)},
+        "e2e": {"value": round(world * bytes_step / (e2e_step_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_step_ms, 5), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "api": "paged_kv_cache_442_b200.pa_store_kvcache + pa_decode (C ABI) on pinned host buffers"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.headline_only:
+        line["other_workloads"] = measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ct, cb, n, cores, blas = cpu_oracle_time(w)
+        line["cpu_baseline"] = {"value": round(cb / ct / 1e9, 4), "unit": "GB/s", "cores": cores,
+                                "blas_threads": blas, "kind": "oracle",
+                                "sample": f"oracle decode of {n} single sequences of {cfg.name} "
+                                          f"on its own pools ({ct:.1f} s of CPU time)"}
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _rank_workload(cfg, rank):
+    from dataclasses import replace
+    return generate(replace(cfg, index=cfg.index + 100 * rank))
+
+
+def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=200, warmup=10):
+    """Device-timed numbers of the other configurations (same method, fewer steps)."""
+    res = {}
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for name in ("long_ctx_decode", "prefix_share_decode", "chunked_prefill"):
+        w = generate(CONFIGS[name])
+        r = GpuRunner(w, torch, pa)
+        n = steps if w.kind == "decode" else 50
+        total_ms, attn_ms, lps = time_steps(r, torch, n, warmup, flush)
+        a_ms = sum(attn_ms) / len(attn_ms)
+        d = {"attn_us": round(a_ms * 1e3, 2), "step_us": round(total_ms / n * 1e3, 2), "steps": n}
+        if w.kind == "decode":
+            lb = decode_bytes(w)
+            d.update({"kernel": "pa_decode", "logical_bytes": lb, "logical_GBps": round(lb / a_ms / 1e6, 1),
+                      "frac_of_hbm_peak_logical": round(lb / a_ms / 1e6 / hbm_peak, 3),
+                      "partition_size": r.P})
+            if name == "prefix_share_decode":
+                ub = w.kv_bytes_unique() + 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+                d.update({"unique_bytes": ub, "unique_GBps": round(ub / a_ms / 1e6, 1),
+                          "frac_of_hbm_peak_unique": round(ub / a_ms / 1e6 / hbm_peak, 3)})
+        else:
+            fl = prefill_flops(w)
+            st_ms = total_ms / n - a_ms
+            d.update({"kernel": "pa_prefill (tcgen05)", "flops": fl,
+                      "TFLOPs": round(fl / a_ms / 1e9, 1),
+                      "frac_of_bf16_peak_sustained": round(fl / a_ms / 1e9 / tf_sustained, 3),
+                      "frac_of_bf16_peak_burst": round(fl / a_ms / 1e9 / tf_peak, 3),
+                      "store_us": round(st_ms * 1e3, 2),
+                      "store_GBps": round(store_bytes(w) / st_ms / 1e6, 1)})
+        d["peak_source"] = peak_src
+        res[name] = d
+        del r
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_reference(args, cfg, world):
+    """Reference arm: the CPU oracle as it stands, on the host cores. Each step is a
+    bounded sample of the workload: the oracle's decode of 2 of its sequences, on
+    pools the oracle built itself (setup rows and the new tokens already stored)."""
+    w = generate(cfg)
+    pools = oracle_pools_for(w)
+    per_step = 2
+    times, byts = [], []
+    for i in range(args.warmup + args.steps):
+        dt, nb = 0.0, 0
+        for j in range(per_step):
+            a, b = oracle_decode_one(w, pools, (i * per_step + j) % w.num_seqs)
+            dt += a
+            nb += b
+        if i >= args.warmup:
+            times.append(dt)
+            byts.append(nb)
+    tot = sum(times)
+    value = sum(byts) / tot / 1e9
+    cores, blas = host_threads()
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / len(times), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "sample_per_step": f"{per_step} of {w.num_seqs} sequences"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "blas_threads": blas, "kind": "oracle",
+                             "sample": f"oracle decode of {per_step} sequences per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

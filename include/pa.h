@@ -1,0 +1,182 @@
+/*
+ * pa.h — C ABI of the B200 paged KV-cache library (libpa.so).
+ *
+ * The library keeps the keys and values of every sequence in a pre-allocated
+ * pool of fixed-size blocks and reaches them through per-sequence block tables
+ * (nano vllm KV-cache practice page, section 3.2.1 "Block设计" and section 3.1
+ * "Sequence管理": each Sequence owns a block_table; mini-vllm page, section 2
+ * "KVCache": the block table decides where in the pre-allocated GPU tensor K/V
+ * are read and written).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All pointers are DEVICE pointers into memory the caller owns (allocated
+ *    by the caller, e.g. through PyTorch). The library allocates no device
+ *    memory and keeps no per-call state; scratch space is passed in.
+ *  - bf16 tensors are dense, row-major, 16-byte aligned.
+ *  - Pool layout (k_cache, v_cache): [num_blocks, block_size, num_kv_heads,
+ *    head_dim] bf16. Logical position p of sequence s lives in pool row
+ *        block_tables[s * max_blocks_per_seq + p / block_size] * block_size
+ *        + p % block_size,
+ *    a row being num_kv_heads * head_dim contiguous bf16 values.
+ *  - block_tables: int32 [num_seqs, max_blocks_per_seq], unused entries -1.
+ *  - context_lens: int32 [num_seqs], the number of positions of each sequence
+ *    INCLUDING the tokens written in the current step.
+ *  - Grouped-query attention: query head h reads kv head
+ *    h / (num_q_heads / num_kv_heads).
+ *  - Scores are scale * dot(q, k); softmax over the visible positions; the
+ *    result is rounded once to bf16 (nearest even). Accumulation is fp32.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and do not synchronise, except when debug checks are on
+ *    (see pa_set_debug_checks).
+ *
+ * Errors
+ * ------
+ *  - Arguments are validated on the host before any launch; a bad argument
+ *    returns PA_ERR_INVALID_ARG and launches nothing. Supported sizes:
+ *    head_dim 64 or 128; block_size a power of two in [16, 1024];
+ *    num_q_heads a multiple of num_kv_heads.
+ *  - A valid but unimplemented combination returns PA_ERR_UNSUPPORTED.
+ *  - A failed launch returns PA_ERR_CUDA.
+ *  - Device-side index checks never trap: an out-of-range block id or slot is
+ *    recorded in a device error word and the access is redirected to row 0 of
+ *    the pool (store: the write is skipped). The error word is read (and
+ *    cleared) by pa_check_device_errors, which returns PA_ERR_BAD_INDEX, or
+ *    PA_ERR_TIMEOUT if a bounded wait inside a kernel gave up.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_BAD_INDEX = 3,
+  PA_ERR_CUDA = 4,
+  PA_ERR_TIMEOUT = 5
+} pa_status;
+
+/* Shape of the paged pool (both k_cache and v_cache have this shape). */
+typedef struct {
+  int32_t num_blocks;   /* physical blocks in the pool                     */
+  int32_t block_size;   /* token positions per block (power of two)        */
+  int32_t num_kv_heads; /* Hkv                                             */
+  int32_t head_dim;     /* D: 64 or 128                                    */
+} pa_cache_desc;
+
+/*
+ * pa_store_kvcache — write the K/V rows of this step's new tokens into the pool.
+ *
+ * Defines: k_cache[slot_mapping[t]] = k[t] and v_cache[slot_mapping[t]] = v[t]
+ * for every t with slot_mapping[t] >= 0 (mini-vllm page, section 2: the block
+ * table decides where K/V are written; the caller turns (sequence, position)
+ * into a pool row ("slot") with the row formula above).
+ *
+ *   k, v          [num_tokens, Hkv, D] bf16, read only.
+ *   k_cache,
+ *   v_cache       pool, written in place (only the mapped rows change).
+ *   slot_mapping  int32 [num_tokens]; -1 skips the token. Two tokens mapped to
+ *                 one slot is a caller error (the surviving row is unspecified).
+ *   num_tokens    >= 0; 0 is a no-op.
+ * A slot >= num_blocks * block_size is skipped and flags PA_ERR_BAD_INDEX.
+ */
+pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
+                           pa_cache_desc cache, const int32_t* slot_mapping,
+                           int32_t num_tokens, void* stream);
+
+/*
+ * Decode split size. The context of every sequence is cut into partitions of
+ * partition_size positions (a multiple of 64); each (sequence, kv head,
+ * partition) is processed independently and partials are merged by a second
+ * kernel. pa_decode_default_partition returns the size pa_decode picks when
+ * given partition_size = 0 (depends on the batch, heads, max context and the
+ * device's SM count of the current device).
+ */
+int32_t pa_decode_default_partition(int32_t num_seqs, int32_t num_kv_heads,
+                                    int32_t max_context_len);
+
+/* Bytes of scratch pa_decode needs for these sizes (0 if no split happens). */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size);
+
+/*
+ * pa_decode — one query token per sequence attends over its whole paged
+ * context (mini-vllm page, "性能评估与基准测试": in the decode phase only the one
+ * new token is computed; its K/V must already be stored, so context_lens[s]
+ * counts it).
+ *
+ *   out            [num_seqs, Hq, D] bf16, written.
+ *   q              [num_seqs, Hq, D] bf16.
+ *   block_tables   int32 [num_seqs, max_blocks_per_seq].
+ *   context_lens   int32 [num_seqs]; a sequence with length <= 0 gets zeros.
+ *   scale          softmax scale (1/sqrt(D) for standard attention).
+ *   max_context_len  host upper bound of context_lens (sizes the split); a
+ *                  larger device value is clipped to it and flags
+ *                  PA_ERR_BAD_INDEX.
+ *   partition_size 0 = automatic, else a multiple of 64.
+ *   workspace      device scratch of at least pa_decode_workspace_size(...)
+ *                  bytes (may be NULL when that size is 0); its contents on
+ *                  entry do not matter.
+ * Supported: Hq / Hkv in {1, 2, 4, 8}.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    pa_cache_desc cache, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
+                    int32_t num_q_heads, float scale, int32_t max_context_len,
+                    int32_t partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * pa_prefill — causal attention of a chunk of new tokens appended to each
+ * sequence's cached prefix (nano vllm page, section 3.1: num_cached_tokens of a
+ * Sequence are reused; mini-vllm page, section 1: blocks are allocated for the
+ * prefill). The new tokens' K/V must already be in the pool
+ * (pa_store_kvcache), so every K/V read goes through the block table.
+ *
+ *   out, q         [total_q, Hq, D] bf16 (varlen: sequence s owns rows
+ *                  cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1).
+ *   total_q        rows of q and out (= cu_seqlens_q[num_seqs]); q is never
+ *                  read past it.
+ *   cu_seqlens_q   int32 [num_seqs + 1], non-decreasing, cu_seqlens_q[0] = 0.
+ *   context_lens   int32 [num_seqs]; new token i of sequence s sits at position
+ *                  context_lens[s] - n_new + i and sees positions 0..that one.
+ *                  Requires n_new <= context_lens[s].
+ *   max_q_len      host upper bound of the new tokens of one sequence.
+ * Uses the tcgen05 tensor cores; head_dim must be 128.
+ */
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     pa_cache_desc cache, const int32_t* block_tables,
+                     int32_t max_blocks_per_seq, const int32_t* cu_seqlens_q,
+                     const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                     int32_t total_q, int32_t max_q_len, float scale, void* stream);
+
+/*
+ * Debug mode: when on, every entry point synchronises its stream after the
+ * launch and returns the device error status (see pa_check_device_errors).
+ */
+void pa_set_debug_checks(int on);
+
+/*
+ * Synchronise `stream`, read and clear this device's error word.
+ * Returns PA_OK, PA_ERR_BAD_INDEX, PA_ERR_TIMEOUT or PA_ERR_CUDA.
+ */
+pa_status pa_check_device_errors(void* stream);
+
+/* Human-readable name of a status (static string). */
+const char* pa_status_string(pa_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

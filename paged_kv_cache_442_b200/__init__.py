@@ -1,0 +1,227 @@
+"""Python binding of libpa.so, the B200 paged KV-cache library.
+
+Argument marshalling only: every function here checks tensor dtypes/devices,
+turns torch tensors into device pointers and calls the C entry point of the same
+name (declared in include/pa.h). All arithmetic runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback. If libpa.so is missing or cannot be
+loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libpa.so")
+
+PA_OK = 0
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_BAD_INDEX",
+                4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT"}
+
+# every extern "C" function include/pa.h declares
+EXPORTED = ("pa_store_kvcache", "pa_decode_default_partition", "pa_decode_workspace_size",
+            "pa_decode", "pa_prefill", "pa_set_debug_checks", "pa_check_device_errors",
+            "pa_status_string", "pa_version")
+
+
+class PAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+class pa_cache_desc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Load libpa.so (once). Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not found: build it with `python -m paged_kv_cache_442_b200.build`"
+                          " (the CUDA library is required; there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.pa_store_kvcache.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp]
+    lib.pa_store_kvcache.restype = ctypes.c_int
+    lib.pa_decode_default_partition.argtypes = [i32, i32, i32]
+    lib.pa_decode_default_partition.restype = i32
+    lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.pa_decode_workspace_size.restype = sz
+    lib.pa_decode.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32, ctypes.c_float,
+                              i32, i32, vp, sz, vp]
+    lib.pa_decode.restype = ctypes.c_int
+    lib.pa_prefill.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, vp, i32, i32, i32, i32,
+                               ctypes.c_float, vp]
+    lib.pa_prefill.restype = ctypes.c_int
+    lib.pa_set_debug_checks.argtypes = [ctypes.c_int]
+    lib.pa_set_debug_checks.restype = None
+    lib.pa_check_device_errors.argtypes = [vp]
+    lib.pa_check_device_errors.restype = ctypes.c_int
+    lib.pa_status_string.argtypes = [ctypes.c_int]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------------- marshalling
+def _torch():
+    import torch
+    return torch
+
+
+def _check(t, name, dtype, ndim=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() else ctypes.c_void_p(0)
+
+
+def _raise(fn, status):
+    if status != PA_OK:
+        raise PAError(fn, status)
+
+
+def cache_desc(k_cache) -> pa_cache_desc:
+    """Pool shape [num_blocks, block_size, num_kv_heads, head_dim] as the C struct."""
+    nb, bs, hkv, d = k_cache.shape
+    return pa_cache_desc(nb, bs, hkv, d)
+
+
+# ----------------------------------------------------------------- entry points
+def pa_store_kvcache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """k_cache[slot_mapping[t]] = k[t], v_cache[...] = v[t] (slot -1 skips)."""
+    torch = _torch()
+    lib = load_library()
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(slot_mapping, "slot_mapping", torch.int32, 1)
+    if k.shape != v.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("k/v and k_cache/v_cache shapes must match")
+    if k.shape[0] != slot_mapping.shape[0] or tuple(k.shape[1:]) != tuple(k_cache.shape[2:]):
+        raise ValueError("k must be [num_tokens, num_kv_heads, head_dim] matching the pool")
+    st = lib.pa_store_kvcache(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+                              _ptr(slot_mapping), int(k.shape[0]), _stream(stream))
+    _raise("pa_store_kvcache", st)
+
+
+def pa_decode_default_partition(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:
+    return int(load_library().pa_decode_default_partition(num_seqs, num_kv_heads, max_context_len))
+
+
+def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                             partition_size: int) -> int:
+    return int(load_library().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+                                                       max_context_len, partition_size))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+              max_context_len: int, partition_size: int = 0, workspace=None, stream=None) -> None:
+    """Paged decode attention into `out` [num_seqs, Hq, D] (bf16)."""
+    torch = _torch()
+    lib = load_library()
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    if tuple(out.shape) != (B, Hq, D) or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("out/q/block_tables/context_lens disagree on num_seqs")
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+                       _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), int(B),
+                       int(Hq), float(scale), int(max_context_len), int(partition_size),
+                       _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
+                       _stream(stream))
+    _raise("pa_decode", st)
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, cu_seqlens_q, context_lens, scale: float,
+               max_q_len: int, stream=None) -> None:
+    """Causal paged prefill into `out` [total_q, Hq, D] (bf16)."""
+    torch = _torch()
+    lib = load_library()
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    Tq, Hq, D = q.shape
+    B = context_lens.shape[0]
+    if tuple(out.shape) != (Tq, Hq, D) or cu_seqlens_q.shape[0] != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("out/q/cu_seqlens_q/block_tables/context_lens shapes disagree")
+    st = lib.pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+                        _ptr(block_tables), int(block_tables.shape[1]), _ptr(cu_seqlens_q),
+                        _ptr(context_lens), int(B), int(Hq), int(Tq), int(max_q_len), float(scale),
+                        _stream(stream))
+    _raise("pa_prefill", st)
+
+
+def pa_set_debug_checks(on: bool) -> None:
+    load_library().pa_set_debug_checks(1 if on else 0)
+
+
+def pa_check_device_errors(stream=None) -> int:
+    """Synchronise, read and clear the device error word; returns a status code."""
+    return int(load_library().pa_check_device_errors(_stream(stream)))
+
+
+def pa_status_string(status: int) -> str:
+    return load_library().pa_status_string(int(status)).decode()
+
+
+def pa_version() -> int:
+    return int(load_library().pa_version())
+
+
+def decode_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                     partition_size=0, device="cuda"):
+    """Allocate (with torch) the scratch pa_decode needs.
+
+    Returns (workspace tensor or None, partition size); pass both to pa_decode so
+    the split it runs is the one the scratch was sized for.
+    """
+    torch = _torch()
+    P = partition_size or pa_decode_default_partition(num_seqs, num_kv_heads, max_context_len)
+    nbytes = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, P)
+    if nbytes == 0:
+        return None, P
+    return torch.empty(nbytes // 4, dtype=torch.float32, device=device), P

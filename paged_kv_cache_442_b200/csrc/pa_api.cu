@@ -1,0 +1,298 @@
+// C ABI of libpa.so: argument validation, scratch-space sizing, device error
+// word and tensor-map encoding. Kernels live in store_kvcache.cu, decode.cu and
+// prefill.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace pa {
+
+// One word per device that loads the library: bit 0 = bad index, bit 1 = timeout.
+__device__ unsigned g_device_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_debug{0};
+std::mutex g_mu;
+unsigned* g_err_ptr[kMaxDevices] = {nullptr};
+int g_sm_count[kMaxDevices] = {0};
+std::set<std::pair<const void*, int>> g_smem_set;  // (kernel, device) already raised
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+pa_status check_cache(const pa_cache_desc& c) {
+  if (c.num_blocks <= 0 || c.num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (!is_pow2(c.block_size) || c.block_size < 16 || c.block_size > 1024) return PA_ERR_INVALID_ARG;
+  if (c.head_dim != 64 && c.head_dim != 128) return PA_ERR_INVALID_ARG;
+  const int64_t slots = static_cast<int64_t>(c.num_blocks) * c.block_size;
+  if (slots > INT32_MAX) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+pa_status finish(cudaError_t e, void* stream) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // clear a sticky launch error from the runtime's slot
+    return e == cudaErrorInvalidValue ? PA_ERR_INVALID_ARG : PA_ERR_CUDA;
+  }
+  if (g_debug.load(std::memory_order_relaxed)) return pa_check_device_errors(stream);
+  return PA_OK;
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+unsigned* device_error_word() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[d]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[d] = static_cast<unsigned*>(ptr);
+  }
+  return g_err_ptr[d];
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sm_count[d]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[d] = n;
+  }
+  return g_sm_count[d];
+}
+
+cudaError_t ensure_max_dynamic_smem(const void* func, int bytes) {
+  const int d = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto key = std::make_pair(func, d);
+  if (g_smem_set.count(key)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) g_smem_set.insert(key);
+  return e;
+}
+
+bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1,
+                          uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
+                          bool swizzle128) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  }
+  const cuuint64_t dims[3] = {dim0, dim1, dim2};
+  const cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {box0, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int32_t pa_version(void) { return 100; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_BAD_INDEX: return "PA_ERR_BAD_INDEX";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+void pa_set_debug_checks(int on) { g_debug.store(on ? 1 : 0); }
+
+pa_status pa_check_device_errors(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  unsigned* w = device_error_word();
+  if (!w) return PA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return PA_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  if (v & PA_DEV_ERR_TIMEOUT) return PA_ERR_TIMEOUT;
+  if (v & PA_DEV_ERR_BAD_INDEX) return PA_ERR_BAD_INDEX;
+  return PA_OK;
+}
+
+pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
+                           pa_cache_desc cache, const int32_t* slot_mapping, int32_t num_tokens,
+                           void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  return finish(launch_store_kvcache(k, v, k_cache, v_cache, cache, slot_mapping, num_tokens,
+                                     static_cast<cudaStream_t>(stream)),
+                stream);
+}
+
+int32_t pa_decode_default_partition(int32_t num_seqs, int32_t num_kv_heads,
+                                    int32_t max_context_len) {
+  // Split until the grid has enough (sequence, kv head, partition) CTAs to keep
+  // every SM busy for several waves, but never below 256 positions, and cap a
+  // partition at 2048 so that uneven lengths do not leave a long tail.
+  const int64_t units = static_cast<int64_t>(num_seqs > 0 ? num_seqs : 1) *
+                        (num_kv_heads > 0 ? num_kv_heads : 1);
+  const int64_t want = static_cast<int64_t>(sm_count()) * 8;
+  int P = round_up(max_context_len > 64 ? max_context_len : 64, 64);
+  if (P > 2048) P = 2048;
+  while (P > 256 && units * ((max_context_len + P - 1) / P) < want) P = round_up(P / 2, 64);
+  return P;
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  if (partition_size <= 0) return 0;
+  const int64_t parts = (max_context_len + partition_size - 1) / partition_size;
+  if (parts <= 1) return 0;
+  return static_cast<size_t>(num_seqs) * num_q_heads * parts * (head_dim + 2) * sizeof(float);
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    pa_cache_desc cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                    float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache.num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) >
+      static_cast<int64_t>(max_blocks_per_seq) * cache.block_size)
+    return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache.num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (partition_size < 0 || (partition_size % 64) != 0) return PA_ERR_INVALID_ARG;
+  const int P = partition_size > 0 ? partition_size
+                                   : pa_decode_default_partition(num_seqs, cache.num_kv_heads,
+                                                                 max_context_len);
+  const int parts = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
+  const size_t need =
+      pa_decode_workspace_size(num_seqs, num_q_heads, cache.head_dim, max_context_len, P);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+
+  DecodeLaunch a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cache = cache;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.scale = scale;
+  a.max_context_len = max_context_len;
+  a.partition_size = P;
+  a.max_parts = parts;
+  float* ws = static_cast<float*>(workspace);
+  a.ws_o = need ? ws : nullptr;
+  a.ws_ml = need ? ws + static_cast<size_t>(num_seqs) * num_q_heads * parts * cache.head_dim
+                 : nullptr;
+  return finish(launch_decode(a, static_cast<cudaStream_t>(stream)), stream);
+}
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     pa_cache_desc cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* cu_seqlens_q, const int32_t* context_lens, int32_t num_seqs,
+                     int32_t num_q_heads, int32_t total_q, int32_t max_q_len, float scale,
+                     void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || total_q < 0 ||
+      max_q_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache.num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (cache.head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_seqlens_q || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  PrefillLaunch a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cache = cache;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.cu_seqlens_q = cu_seqlens_q;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.max_q_len = max_q_len;
+  a.total_q = total_q;
+  a.scale = scale;
+  return finish(launch_prefill(a, static_cast<cudaStream_t>(stream)), stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Internal host-side interfaces between the C ABI layer (pa_api.cu) and the
+// kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// Bits of the per-device error word that kernels set instead of trapping.
+constexpr unsigned PA_DEV_ERR_BAD_INDEX = 1u;
+constexpr unsigned PA_DEV_ERR_TIMEOUT = 2u;
+
+// Per-device pointer to the device error word (lives in pa_api.cu).
+unsigned* device_error_word();
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_max_dynamic_smem(const void* func, int bytes);
+
+// Encode a 3-D bf16 tensor map over a [dim2][dim1][dim0] row-major tensor.
+// swizzle128: 128-byte swizzle (box_dim0 * 2 must then be <= 128).
+bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1,
+                          uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
+                          bool swizzle128);
+
+cudaError_t launch_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
+                                 const pa_cache_desc& c, const int32_t* slot_mapping,
+                                 int32_t num_tokens, cudaStream_t stream);
+
+struct DecodeLaunch {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  pa_cache_desc cache;
+  const int32_t* block_tables;
+  int32_t max_blocks_per_seq;
+  const int32_t* context_lens;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  float scale;
+  int32_t max_context_len;
+  int32_t partition_size;  // resolved (> 0)
+  int32_t max_parts;       // ceil(max_context_len / partition_size)
+  float* ws_o;             // [B, Hq, max_parts, D] fp32 (NULL when max_parts == 1)
+  float* ws_ml;            // [B, Hq, max_parts, 2] fp32
+};
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+
+struct PrefillLaunch {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  pa_cache_desc cache;
+  const int32_t* block_tables;
+  int32_t max_blocks_per_seq;
+  const int32_t* cu_seqlens_q;
+  const int32_t* context_lens;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t max_q_len;
+  int32_t total_q;  // rows of q/out (cu_seqlens_q[num_seqs]) upper bound for the tensor map
+  float scale;
+};
+cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,123 @@
+"""The C ABI library loads, exports every function include/pa.h declares, and its
+host-side validation rejects bad arguments before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_442_b200 as pa
+from paged_kv_cache_442_b200 import build as pa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(pa.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (pa_\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_host_only_calls(lib):
+    assert pa.pa_version() == 100
+    assert pa.pa_status_string(0) == "PA_OK"
+    assert pa.pa_status_string(5) == "PA_ERR_TIMEOUT"
+    # workspace: [B, Hq, parts, D + 2] fp32 when the context is split, else nothing
+    assert pa.pa_decode_workspace_size(8, 32, 128, 32768, 1024) == 8 * 32 * 32 * 130 * 4
+    assert pa.pa_decode_workspace_size(8, 32, 128, 1024, 1024) == 0
+    assert pa.pa_decode_workspace_size(0, 32, 128, 1024, 256) == 0
+
+
+def desc(nb=16, bs=16, hkv=2, d=128):
+    return pa.pa_cache_desc(nb, bs, hkv, d)
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("bad", [desc(bs=12), desc(bs=8), desc(bs=2048), desc(d=96), desc(nb=0),
+                                 desc(hkv=0), desc(nb=1 << 22, bs=1024)])
+def test_bad_cache_shapes_are_rejected(lib, bad):
+    st = lib.pa_store_kvcache(FAKE, FAKE, FAKE, FAKE, bad, FAKE, 4, NULL)
+    assert st == 1
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, bad, FAKE, 4, FAKE, 2, 4, 0.1, 32, 0, NULL, 0, NULL)
+    assert st == 1
+
+
+def test_store_argument_checks(lib):
+    assert lib.pa_store_kvcache(NULL, FAKE, FAKE, FAKE, desc(), FAKE, 4, NULL) == 1
+    assert lib.pa_store_kvcache(FAKE, FAKE, FAKE, FAKE, desc(), FAKE, -1, NULL) == 1
+    misaligned = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.pa_store_kvcache(misaligned, FAKE, FAKE, FAKE, desc(), FAKE, 4, NULL) == 1
+    assert lib.pa_store_kvcache(NULL, NULL, NULL, NULL, desc(), NULL, 0, NULL) == 0  # no-op
+
+
+def test_decode_argument_checks(lib):
+    d = desc(hkv=2)
+    # Hq not a multiple of Hkv
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 3, 0.1, 32, 0, NULL, 0, NULL) == 1
+    # group of 3 query heads per kv head: valid but not implemented
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 6, 0.1, 32, 0, NULL, 0, NULL) == 2
+    # context longer than the block table can address
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 65, 0, NULL, 0, NULL) == 1
+    # non-finite scale
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, float("nan"), 32, 0, NULL, 0,
+                         NULL) == 1
+    # partition size not a multiple of 64
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 32, 100, NULL, 0, NULL) == 1
+    # split needs a workspace
+    assert lib.pa_decode(FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 64, 64, NULL, 0, NULL) == 1
+    # empty batch is a no-op
+    assert lib.pa_decode(NULL, NULL, NULL, NULL, d, NULL, 4, NULL, 0, 4, 0.1, 32, 0, NULL, 0, NULL) == 0
+
+
+def test_prefill_argument_checks(lib):
+    assert lib.pa_prefill(FAKE, FAKE, FAKE, FAKE, desc(d=64), FAKE, 4, FAKE, FAKE, 2, 4, 8, 4, 0.1,
+                          NULL) == 2
+    assert lib.pa_prefill(FAKE, FAKE, FAKE, FAKE, desc(), FAKE, 4, FAKE, FAKE, 2, 3, 8, 4, 0.1,
+                          NULL) == 1
+    assert lib.pa_prefill(NULL, FAKE, FAKE, FAKE, desc(), FAKE, 4, FAKE, FAKE, 2, 4, 8, 4, 0.1,
+                          NULL) == 1
+    assert lib.pa_prefill(NULL, NULL, NULL, NULL, desc(), NULL, 4, NULL, NULL, 2, 4, 0, 0, 0.1,
+                          NULL) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    k = torch.zeros(4, 2, 128, dtype=torch.bfloat16)
+    cache = torch.zeros(16, 16, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_store_kvcache(k, k, cache, cache, torch.zeros(4, dtype=torch.int32))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import importlib
+    saved = pa._lib
+    try:
+        pa._lib = None
+        with pytest.raises(ImportError, match="no CPU fallback"):
+            pa.load_library(str(tmp_path / "nope.so"))
+    finally:
+        pa._lib = saved
