@@ -414,6 +414,22 @@ def main():
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
+    if w.kind == "decode":
+        roofline = {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
+                    "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                    "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
+                    "algorithmic_bytes_per_launch": attn_bytes,
+                    "avg_launch_us": round(attn_avg_ms * 1e3, 2),
+                    "traffic": recorded_traffic(cfg.name + ".decode", DECODE_SRC)}
+    else:
+        fl = prefill_flops(w)
+        tf = fl / (attn_avg_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "pa_prefill (tcgen05)", "achieved": round(tf, 1),
+                    "peak": tf_peak, "unit": "TFLOP/s", "frac": round(tf / tf_peak, 3),
+                    "frac_of_sustained": round(tf / tf_sustained, 3),
+                    "peak_source": f"{peak_src} bf16 GEMM (burst)",
+                    "algorithmic_flops_per_launch": fl, "avg_launch_us": round(attn_avg_ms * 1e3, 2),
+                    "traffic": recorded_traffic(cfg.name + ".prefill", PREFILL_SRC)}
 
     e2e_ms, h2d, d2h = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
     e2e_step_ms = e2e_ms / min(args.steps, 500)
@@ -442,12 +458,7 @@ def main():
         "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
         "pct_of_datasheet_8tbs": round(100 * value / world / DATASHEET_HBM_GBS, 1),
         "bytes_per_step": bytes_step,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
-                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
-                     "algorithmic_bytes_per_launch": attn_bytes,
-                     "avg_launch_us": round(attn_avg_ms * 1e3, 2),
-                     "traffic": recorded_traffic(cfg.name + ".decode", DECODE_SRC)},
+        "roofline": roofline,
         "e2e": {"value": round(world * bytes_step / (e2e_step_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_step_ms, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,

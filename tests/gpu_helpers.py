@@ -9,8 +9,16 @@ import oracle
 import paged_kv_cache_442_b200 as pa
 from workloads import SENTINEL_BF16
 
-TOL_ABS = 1e-2   # max |gpu - oracle|
-TOL_REL = 1e-2   # ||gpu - oracle||_2 / ||oracle||_2
+# Parity bar ("max abs error 1e-2 with relative error 1e-2 on bf16 outputs"):
+#   per element |g - r| <= TOL_ABS + TOL_REL * |r|   (the abs+rel "allclose" form: a
+#     bf16 output of magnitude >= 4 is already up to 2**-6 = 0.0156 away from the exact
+#     value after its one mandated rounding, so a bare 1e-2 absolute bound would reject
+#     correctly rounded results), and
+#   over the whole tensor ||g - r||_2 / ||r||_2 <= TOL_NORM (keeps the check meaningful
+#     at long context, where outputs are ~1e-2 and the element bound alone is loose).
+TOL_ABS = 1e-2
+TOL_REL = 1e-2
+TOL_NORM = 1e-2
 
 
 def bf16_dev(bits: np.ndarray) -> torch.Tensor:
@@ -101,5 +109,9 @@ def oracle_prefill(w, pools=None):
 def assert_close(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
     c = oracle.compare(gpu, ref)
     assert c["finite"], f"{what}: non-finite GPU output"
-    assert c["max_abs"] <= TOL_ABS and c["norm_rel"] <= TOL_REL, f"{what}: {c}"
+    g = np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    excess = np.abs(g - r) - (TOL_ABS + TOL_REL * np.abs(r))
+    c["worst_excess"] = float(excess.max()) if excess.size else 0.0
+    assert c["worst_excess"] <= 0.0 and c["norm_rel"] <= TOL_NORM, f"{what}: {c}"
     return c
