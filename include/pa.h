@@ -134,6 +134,39 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * pa_decode_no_alloc — pa_decode for callers that cannot allocate device memory.
+ * (The pages have no counterpart: this is an interface convenience, not a step of
+ * the method.)
+ *
+ * Some callers have no way to provide pa_decode's workspace: a serving runtime
+ * that carves the GPU into fixed pools at start-up and allows no allocation
+ * afterwards, or a host program that drives this library only through its C ABI
+ * without access to a CUDA allocator. This entry point takes the same arguments
+ * as pa_decode minus the workspace, and uses instead a scratch array of
+ * PA_DECODE_NO_ALLOC_SCRATCH_BYTES that the library owns: a device array that
+ * every GPU loading the library holds until the process exits. It allocates
+ * nothing and calls no allocator. The caller still passes inputs and outputs.
+ *
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current), which may load the
+ *    library's device code; make that first call before any stream capture.
+ *  - Sizes whose split-K scratch (pa_decode_workspace_size for the partition
+ *    used) exceeds PA_DECODE_NO_ALLOC_SCRATCH_BYTES are rejected with
+ *    PA_ERR_UNSUPPORTED and nothing is launched; pass a larger partition_size
+ *    or use pa_decode.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents; nothing in it has to start at zero (each partial is written
+ *    before it is read). Calls that overlap on the GPU (e.g. on two streams
+ *    without ordering between them) race on the array: order them.
+ */
+#define PA_DECODE_NO_ALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             pa_cache_desc cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t num_q_heads, float scale,
+                             int32_t max_context_len, int32_t partition_size, void* stream);
+
+/*
  * pa_prefill — causal attention of a chunk of new tokens appended to each
  * sequence's cached prefix (nano vllm page, section 3.1: num_cached_tokens of a
  * Sequence are reused; mini-vllm page, section 1: blocks are allocated for the

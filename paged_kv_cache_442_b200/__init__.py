@@ -20,8 +20,11 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
 
 # every extern "C" function include/pa.h declares
 EXPORTED = ("pa_store_kvcache", "pa_decode_default_partition", "pa_decode_workspace_size",
-            "pa_decode", "pa_prefill", "pa_set_debug_checks", "pa_check_device_errors",
-            "pa_status_string", "pa_version")
+            "pa_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
+            "pa_check_device_errors", "pa_status_string", "pa_version")
+
+# size of the library-owned scratch of pa_decode_no_alloc (include/pa.h)
+DECODE_NO_ALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 class PAError(RuntimeError):
@@ -58,6 +61,9 @@ def load_library(path: str | None = None):
     lib.pa_decode.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32, ctypes.c_float,
                               i32, i32, vp, sz, vp]
     lib.pa_decode.restype = ctypes.c_int
+    lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
+                                       ctypes.c_float, i32, i32, vp]
+    lib.pa_decode_no_alloc.restype = ctypes.c_int
     lib.pa_prefill.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, vp, i32, i32, i32, i32,
                                ctypes.c_float, vp]
     lib.pa_prefill.restype = ctypes.c_int
@@ -170,6 +176,40 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                        _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
                        _stream(stream))
     _raise("pa_decode", st)
+
+
+def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                       max_context_len: int, partition_size: int = 0, stream=None) -> None:
+    """pa_decode for callers that cannot allocate device memory.
+
+    Same result as pa_decode, but the split-K scratch is a fixed array the library
+    owns (DECODE_NO_ALLOC_SCRATCH_BYTES per GPU), so the caller passes no
+    workspace and nothing is allocated. Sizes that need more scratch than that are
+    rejected; calls on one GPU share the array, so they must not overlap.
+    """
+    torch = _torch()
+    lib = load_library()
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    if tuple(out.shape) != (B, Hq, D) or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("out/q/block_tables/context_lens disagree on num_seqs")
+    st = lib.pa_decode_no_alloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                cache_desc(k_cache), _ptr(block_tables), int(block_tables.shape[1]),
+                                _ptr(context_lens), int(B), int(Hq), float(scale),
+                                int(max_context_len), int(partition_size), _stream(stream))
+    if st == 2:
+        P = partition_size or pa_decode_default_partition(B, k_cache.shape[2], max_context_len)
+        need = pa_decode_workspace_size(B, Hq, D, max_context_len, P)
+        if need > DECODE_NO_ALLOC_SCRATCH_BYTES:
+            raise PAError(f"pa_decode_no_alloc (needs {need} bytes of split-K scratch, more than "
+                          f"the library's fixed {DECODE_NO_ALLOC_SCRATCH_BYTES}; use a larger "
+                          f"partition_size or pa_decode with a workspace)", st)
+    _raise("pa_decode_no_alloc", st)
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, cu_seqlens_q, context_lens, scale: float,
