@@ -59,7 +59,8 @@ def file_hash(*paths):
     return h.hexdigest()[:16]
 
 
-DECODE_SRC = ("paged_kv_cache_442_b200/csrc/decode.cu", "paged_kv_cache_442_b200/csrc/pa_ptx.cuh")
+DECODE_SRC = ("paged_kv_cache_442_b200/csrc/decode.cu", "paged_kv_cache_442_b200/csrc/decode_tc.cu",
+              "paged_kv_cache_442_b200/csrc/pa_api.cu", "paged_kv_cache_442_b200/csrc/pa_ptx.cuh")
 PREFILL_SRC = ("paged_kv_cache_442_b200/csrc/prefill.cu", "paged_kv_cache_442_b200/csrc/pa_ptx.cuh")
 
 
@@ -230,7 +231,7 @@ def time_steps(runner, torch, steps, warmup, flush_buf, barrier=None):
     stream = torch.cuda.current_stream()
     flush_out = torch.zeros((), dtype=flush_buf.dtype, device=flush_buf.device)
     for _ in range(warmup):
-        torch.sum(flush_buf, out=flush_out)
+        torch.sum(flush_buf, dim=0, out=flush_out)
         runner.step()
     torch.cuda.synchronize()
     if barrier:
@@ -240,7 +241,7 @@ def time_steps(runner, torch, steps, warmup, flush_buf, barrier=None):
            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     launches = 0
     for i in range(steps):
-        torch.sum(flush_buf, out=flush_out)     # read 256 MiB: evicts the previous step from L2
+        torch.sum(flush_buf, dim=0, out=flush_out)     # read 256 MiB: evicts the previous step from L2
         a, b, c = ev[i]
         a.record(stream)
         launches += runner.store()
@@ -416,7 +417,7 @@ def main():
     attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     if w.kind == "decode":
-        roofline = {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
+        roofline = {"bound": "hbm", "kernel": "pa_decode (persistent tcgen05 decode, split-K merge fused)",
                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                     "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
                     "algorithmic_bytes_per_launch": attn_bytes,

@@ -102,7 +102,13 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
 int32_t pa_decode_default_partition(int32_t num_seqs, int32_t num_kv_heads,
                                     int32_t max_context_len);
 
-/* Bytes of scratch pa_decode needs for these sizes (0 if no split happens). */
+/*
+ * Bytes of scratch pa_decode needs for these sizes (> 0 whenever num_seqs > 0):
+ * a 256-byte-aligned region of 1 + num_seqs * num_q_heads 64-bit work/arrival
+ * counters, then, when the context is split into more than one partition, the
+ * fp32 partials [num_seqs, Hq, parts, D] and their (max, sum) pairs
+ * [num_seqs, Hq, parts, 2].
+ */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t partition_size);
 
@@ -122,9 +128,14 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *                  PA_ERR_BAD_INDEX.
  *   partition_size 0 = automatic, else a multiple of 64.
  *   workspace      device scratch of at least pa_decode_workspace_size(...)
- *                  bytes (may be NULL when that size is 0); its contents on
- *                  entry do not matter.
- * Supported: Hq / Hkv in {1, 2, 4, 8}.
+ *                  bytes for the partition size used; its contents on entry do
+ *                  not matter (its counters carry a tag unique to each call, so
+ *                  leftovers of earlier calls never count). Calls that overlap
+ *                  on the GPU must use different workspaces.
+ * Supported: Hq / Hkv in {1, 2, 4, 8} (and 16 when head_dim is 128).
+ * head_dim 128 runs the persistent tcgen05 kernel (partition_size a multiple
+ * of 128, at most 2048; other sizes run the CUDA-core kernel); head_dim 64 runs
+ * the CUDA-core kernel.
  */
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     pa_cache_desc cache, const int32_t* block_tables,
@@ -156,8 +167,9 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
  *    or use pa_decode.
  *  - Every call on a device shares the one array and it keeps the last call's
  *    contents; nothing in it has to start at zero (each partial is written
- *    before it is read). Calls that overlap on the GPU (e.g. on two streams
- *    without ordering between them) race on the array: order them.
+ *    before it is read, and the counters carry a tag unique to each call).
+ *    Calls that overlap on the GPU (e.g. on two streams without ordering
+ *    between them) race on the array: order them.
  */
 #define PA_DECODE_NO_ALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -62,8 +62,6 @@ pa_status finish(cudaError_t e, void* stream) {
   return PA_OK;
 }
 
-int round_up(int x, int m) { return (x + m - 1) / m * m; }
-
 }  // namespace
 
 unsigned* device_error_word() {
@@ -185,25 +183,30 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
 
 int32_t pa_decode_default_partition(int32_t num_seqs, int32_t num_kv_heads,
                                     int32_t max_context_len) {
-  // Split until the grid has enough (sequence, kv head, partition) CTAs to keep
-  // every SM busy for several waves, but never below 256 positions, and cap a
-  // partition at 2048 so that uneven lengths do not leave a long tail.
-  const int64_t units = static_cast<int64_t>(num_seqs > 0 ? num_seqs : 1) *
-                        (num_kv_heads > 0 ? num_kv_heads : 1);
-  const int64_t want = static_cast<int64_t>(sm_count()) * 8;
-  int P = round_up(max_context_len > 64 ? max_context_len : 64, 64);
-  if (P > 2048) P = 2048;
-  while (P > 256 && units * ((max_context_len + P - 1) / P) < want) P = round_up(P / 2, 64);
+  // Work items are (partition, sequence, kv head) taken dynamically by one
+  // persistent CTA per SM. Aim for ~16 items per SM on the upper bound of the work
+  // (every sequence at max_context_len) so the last items finish close together,
+  // with partitions a power of two in [256, 2048] positions (tiles are 128).
+  const int64_t work = static_cast<int64_t>(num_seqs > 0 ? num_seqs : 1) *
+                       (num_kv_heads > 0 ? num_kv_heads : 1) *
+                       (max_context_len > 0 ? max_context_len : 1);
+  const int64_t per_item = work / (static_cast<int64_t>(sm_count()) * 16);
+  int P = 256;
+  while (P < 2048 && P < per_item) P *= 2;
   return P;
 }
 
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t partition_size) {
-  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  // [epoch-tagged counters][partials o: B*Hq*parts*D fp32][partials (m, l): B*Hq*parts*2]
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
   if (partition_size <= 0) return 0;
-  const int64_t parts = (max_context_len + partition_size - 1) / partition_size;
-  if (parts <= 1) return 0;
-  return static_cast<size_t>(num_seqs) * num_q_heads * parts * (head_dim + 2) * sizeof(float);
+  const size_t counters = decode_counter_bytes(num_seqs, num_q_heads);
+  const int64_t parts =
+      max_context_len > 0 ? (max_context_len + partition_size - 1) / partition_size : 1;
+  if (parts <= 1) return counters;
+  return counters +
+         static_cast<size_t>(num_seqs) * num_q_heads * parts * (head_dim + 2) * sizeof(float);
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -221,7 +224,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
       static_cast<int64_t>(max_blocks_per_seq) * cache.block_size)
     return PA_ERR_INVALID_ARG;
   const int G = num_q_heads / cache.num_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && !(G == 16 && cache.head_dim == 128))
+    return PA_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;
@@ -231,11 +235,13 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   const int P = partition_size > 0 ? partition_size
                                    : pa_decode_default_partition(num_seqs, cache.num_kv_heads,
                                                                  max_context_len);
-  const int parts = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
+  const int64_t parts64 = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
+  // work items are counted in 24 bits, with room for one extra take per CTA
+  if (parts64 * num_seqs * cache.num_kv_heads >= (1ll << 24) - 4096) return PA_ERR_UNSUPPORTED;
+  const int parts = static_cast<int>(parts64);
   const size_t need =
       pa_decode_workspace_size(num_seqs, num_q_heads, cache.head_dim, max_context_len, P);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-    return PA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
 
   DecodeLaunch a;
   a.out = out;
@@ -252,11 +258,16 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.max_context_len = max_context_len;
   a.partition_size = P;
   a.max_parts = parts;
-  float* ws = static_cast<float*>(workspace);
-  a.ws_o = need ? ws : nullptr;
-  a.ws_ml = need ? ws + static_cast<size_t>(num_seqs) * num_q_heads * parts * cache.head_dim
-                 : nullptr;
-  return finish(launch_decode(a, static_cast<cudaStream_t>(stream)), stream);
+  const size_t cbytes = decode_counter_bytes(num_seqs, num_q_heads);
+  unsigned long long* counters = static_cast<unsigned long long*>(workspace);
+  float* ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
+  a.ws_o = parts > 1 ? ws : nullptr;
+  a.ws_ml = parts > 1 ? ws + static_cast<size_t>(num_seqs) * num_q_heads * parts * cache.head_dim
+                      : nullptr;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (decode_tc_supported(a)) return finish(launch_decode_tc(a, counters, s), stream);
+  if (G == 16) return PA_ERR_UNSUPPORTED;
+  return finish(launch_decode(a, s), stream);
 }
 
 pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -54,6 +54,18 @@ struct DecodeLaunch {
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 
+// Persistent tcgen05 decode (head dim 128). `counters` is the workspace's counter
+// region: 1 + num_seqs * num_q_heads epoch-tagged 64-bit counters.
+bool decode_tc_supported(const DecodeLaunch& a);
+cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters,
+                             cudaStream_t stream);
+
+// Bytes of the counter region at the start of the decode workspace (256-aligned).
+inline size_t decode_counter_bytes(int32_t num_seqs, int32_t num_q_heads) {
+  const size_t b = 8 * (1 + static_cast<size_t>(num_seqs) * num_q_heads);
+  return (b + 255) / 256 * 256;
+}
+
 struct PrefillLaunch {
   void* out;
   const void* q;

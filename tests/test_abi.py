@@ -43,9 +43,11 @@ def test_host_only_calls(lib):
     assert pa.pa_version() == 100
     assert pa.pa_status_string(0) == "PA_OK"
     assert pa.pa_status_string(5) == "PA_ERR_TIMEOUT"
-    # workspace: [B, Hq, parts, D + 2] fp32 when the context is split, else nothing
-    assert pa.pa_decode_workspace_size(8, 32, 128, 32768, 1024) == 8 * 32 * 32 * 130 * 4
-    assert pa.pa_decode_workspace_size(8, 32, 128, 1024, 1024) == 0
+    # workspace: 256-aligned counters (1 + B*Hq of 8 bytes), then [B, Hq, parts, D + 2]
+    # fp32 partials when the context is split
+    counters = -(-(8 * (1 + 8 * 32)) // 256) * 256
+    assert pa.pa_decode_workspace_size(8, 32, 128, 32768, 1024) == counters + 8 * 32 * 32 * 130 * 4
+    assert pa.pa_decode_workspace_size(8, 32, 128, 1024, 1024) == counters
     assert pa.pa_decode_workspace_size(0, 32, 128, 1024, 256) == 0
 
 
