@@ -110,6 +110,10 @@ struct DecodeSmem {
   static constexpr int kMLOff = kAbufOff + 4 * G * 4;
   static constexpr int kIdsOff = kMLOff + 2 * 4 * G * 4;
   static_assert(4 * G * D * 4 <= kRingBytes, "merge buffer must fit in the ring");
+  static_assert(kTileBytes % 128 == 0 && kStageBytes % 128 == 0, "TMA destinations: 128 B");
+  static_assert(kBarOff % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(kPbufOff % 4 == 0 && kAbufOff % 4 == 0 && kMLOff % 4 == 0 && kIdsOff % 4 == 0,
+                "float / int buffers");
   // + 1 KB so the ring can start on a 1 KB boundary whatever the base alignment
   static int bytes(int max_table_entries) { return kIdsOff + 4 * max_table_entries + 1024; }
 };

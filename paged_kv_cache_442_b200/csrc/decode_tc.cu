@@ -52,9 +52,11 @@ constexpr int NK = 3;          // K ring depth (a slot frees when its score MMA 
 constexpr int NV = 3;          // V ring depth (a slot frees when its value MMA is done)
 constexpr int NS = 4;          // S^T buffers in TMEM
 constexpr int NP = 4;          // P^T buffers in shared memory
-constexpr int QN = 2;          // item queue depth
+constexpr int QN = 2;          // item queue depth (producer -> issuer, softmax)
+constexpr int QS = 2;          // scheduler queue depth: one item prepared ahead (deeper
+                               // queues reserve work early and unbalance the tail)
 constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flight)
-constexpr int kThreads = 320;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9
+constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more than this
 constexpr int kRegion = TM * 128;            // 64 head dims x 128 positions (16 KB)
 constexpr int kTileBytes = 2 * kRegion;      // one K or V tile (32 KB)
@@ -63,19 +65,32 @@ constexpr int kQBytes = 2 * kQRegion;
 constexpr int kPBytes = 2 * kQRegion;        // P^T: 16 heads x 128 positions, bf16
 constexpr int kMaxIds = 2048 / 16 + 2;       // block ids of one item (partition <= 2048)
 
+constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// every region starts on a 16-byte boundary (1024 for the swizzled operand tiles);
+// the static_asserts below keep it that way when depths change
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + NK * kTileBytes;
 constexpr int kOffQ = kOffV + NV * kTileBytes;
 constexpr int kOffP = kOffQ + QN * kQBytes;
-constexpr int kOffRed = kOffP + NP * kPBytes;          // [3][4 warps][NQ] floats
-constexpr int kOffIds = kOffRed + 3 * 4 * NQ * 4;
-constexpr int kOffDesc = kOffIds + 2 * kMaxIds * 4;    // [QN] item descriptors
-constexpr int kOffEpi = kOffDesc + QN * 32;             // [NO] softmax -> epilogue hand-offs
-constexpr int kEpiBytes = 32 + 2 * NQ * 4;              // descriptor, m[NQ], l[NQ]
-constexpr int kOffBar = kOffEpi + NO * kEpiBytes;
-constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO;
-constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kOffRed = kOffP + NP * kPBytes;                     // [3][4 warps][NQ] floats
+constexpr int kOffIds = align_up(kOffRed + 3 * 4 * NQ * 4, 16);
+constexpr int kOffSched = align_up(kOffIds + QS * kMaxIds * 4, 16);  // [QS] descriptors
+constexpr int kOffSchedFb = align_up(kOffSched + QS * 32, 16);       // [QS] first blocks
+constexpr int kOffDesc = align_up(kOffSchedFb + QS * 4, 16);         // [QN] item descriptors
+constexpr int kOffEpi = align_up(kOffDesc + QN * 32, 16);            // [NO] hand-offs
+constexpr int kEpiBytes = 32 + 2 * NQ * 4;                           // descriptor, m, l
+constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
+constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS;
+constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
+              "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
+static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "tile sizes");
+static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kOffSched % 16 == 0 && kOffDesc % 16 == 0 && kOffEpi % 16 == 0 && kEpiBytes % 16 == 0,
+              "descriptor slots");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 128;  // S[NS] at 16*i; O[NO] at 64 + 16*i
 constexpr uint32_t kTmemO = 64;
@@ -137,6 +152,28 @@ __device__ __forceinline__ unsigned tagged_fetch_add(unsigned long long* ctr,
   }
   *ok = true;
   return static_cast<unsigned>(old & kCountMask);
+}
+
+// Same contract as tagged_fetch_add for a counter that only a few threads ever touch
+// (the arrivals of one sequence's partitions): add first, and only if the tag was
+// stale try to restart the count under this call's tag. With so few contenders this
+// is one atomic in the common case. Bounded number of attempts.
+__device__ __forceinline__ unsigned tagged_arrive(unsigned long long* ctr, unsigned long long tag,
+                                                  unsigned* err, bool* ok) {
+  for (int it = 0; it < 4096; ++it) {
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    if ((old >> kCountBits) == tag) {
+      *ok = true;
+      return static_cast<unsigned>(old & kCountMask);
+    }
+    if (atomicCAS(ctr, old + 1, (tag << kCountBits) | 1ull) == old + 1) {
+      *ok = true;
+      return 0u;
+    }
+  }
+  flag_error(err, PA_DEV_ERR_TIMEOUT);
+  *ok = false;
+  return 0;
 }
 
 // bounded wait that also gives up once another role has given up
@@ -230,6 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   uint64_t* o_free = o_full + NO;              // [NO] epilogue read O^T -> issuer
   uint64_t* epi_full = o_free + NO;            // [NO] softmax hand-off -> epilogue
   uint64_t* epi_empty = epi_full + NO;         // [NO] epilogue read the hand-off
+  uint64_t* sched_full = epi_empty + NO;       // [QS] scheduler -> producer
+  uint64_t* sched_empty = sched_full + QS;     // [QS] producer done with a queued item
+  ItemDesc* sched_desc = reinterpret_cast<ItemDesc*>(smem + kOffSched);
+  int* sched_fb = reinterpret_cast<int*>(smem + kOffSchedFb);
   ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + kOffDesc);
   int* ids = reinterpret_cast<int*>(smem + kOffIds);
   float* red = reinterpret_cast<float*>(smem + kOffRed);
@@ -268,6 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       mbar_init(&epi_full[i], 1);
       mbar_init(&epi_empty[i], 1);
     }
+    for (int i = 0; i < QS; ++i) {
+      mbar_init(&sched_full[i], 1);
+      mbar_init(&sched_empty[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -280,6 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // lane 0 waits, the warp follows its verdict (keeps the warp's control flow uniform)
+  auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
+    int okw = 0;
+    if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, okw, 0) != 0;
+  };
+
   if (warp == 4) {
     // ======================================================== producer warp
     if (lane == 0) {
@@ -289,80 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     }
     const int rows = bs < TM ? bs : TM;
     const int nbox = TM / rows;
-    // lane 0 waits, the warp follows its verdict (keeps the warp's control flow uniform)
-    auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
-      int okw = 0;
-      if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag) ? 1 : 0;
-      return __shfl_sync(0xffffffffu, okw, 0) != 0;
-    };
-    // Take items until a non-empty one (or the end): decode it and fetch its block ids
-    // into id buffer `which`. Runs while the previous item's tiles are in flight.
-    auto prepare = [&](ItemDesc& d, int& first_blk, int which) {
-      while (true) {
-        unsigned idx = 0;
-        bool ok = true;
-        if (lane == 0) idx = tagged_fetch_add(p.counters, p.tag, p.err, &ok);
-        idx = __shfl_sync(0xffffffffu, idx, 0);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (*abort_flag) ok = false;
-        if (!ok || idx >= p.total_items) {
-          d.stop = 1;
-          d.ntiles = 0;
-          return;
-        }
-        const int g = idx % p.num_kv_heads;
-        const unsigned rr = idx / p.num_kv_heads;
-        const int s = rr % p.num_seqs;
-        const int part = rr / p.num_seqs;
-        int ctx = __ldg(p.context_lens + s);
-        if (ctx > p.max_context_len) {
-          if (lane == 0 && part == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
-          ctx = p.max_context_len;
-        }
-        if (part * p.partition_size >= ctx) {
-          if (part == 0) {  // empty context: a zero output row
-            for (int i = lane; i < G * HD; i += 32)
-              p.out[(static_cast<int64_t>(s) * Hq + g * G) * HD + i] = __float2bfloat16(0.f);
-          }
-          continue;
-        }
-        const int t0 = part * p.partition_size;
-        const int n = min(ctx - t0, p.partition_size);
-        const int ntiles = (n + TM - 1) / TM;
-        first_blk = t0 >> p.bs_log2;
-        const int nb = ((t0 + ntiles * TM - 1) >> p.bs_log2) - first_blk + 1;
-        int* idb = ids + which * kMaxIds;
-        for (int i = lane; i < nb && i < kMaxIds; i += 32) {
-          const int b = first_blk + i;
-          int id = b < p.max_blocks
-                       ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b)
-                       : -1;
-          if (id < 0 || id >= p.num_blocks) {
-            if ((b << p.bs_log2) < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
-            id = 0;  // in-bounds stand-in; positions past ctx are masked
-          }
-          idb[i] = id;
-        }
-        __syncwarp();
-        d.s = s; d.g = g; d.p = part; d.t0 = t0; d.n = n; d.ntiles = ntiles;
-        d.nparts = (ctx + p.partition_size - 1) / p.partition_size;
-        d.stop = 0;
-        return;
-      }
-    };
-    int k = 0;       // items published
+    int q = 0;       // items taken from the scheduler queue
+    int k = 0;       // items published to the issuer / softmax
     unsigned j = 0;  // tiles issued
-    ItemDesc nxt;
-    int nxt_first = 0;
-    int nbuf = 0;
-    prepare(nxt, nxt_first, nbuf);
     while (true) {
-      const ItemDesc cur = nxt;
-      const int first_blk = nxt_first;
-      const int* idc = ids + nbuf * kMaxIds;
+      const int ss = q % QS;
+      if (!wwait(&sched_full[ss], (q / QS) & 1)) break;
+      const ItemDesc cur = sched_desc[ss];
+      const int first_blk = sched_fb[ss];
+      const int* idc = ids + ss * kMaxIds;
       const int slot = k % QN;
-      if (k >= QN && !wwait(&item_empty[slot], ((k / QN) - 1) & 1))
-        break;
+      if (k >= QN && !wwait(&item_empty[slot], ((k / QN) - 1) & 1)) break;
       if (cur.stop) {
         if (lane == 0) {
           descs[slot] = cur;
@@ -380,11 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       }
       bool alive = true;
       for (int i = 0; i < ntiles; ++i, ++j) {
-        if (i == 1 || (i == 0 && ntiles == 1)) {
-          // take the next item while this one's first loads are in flight
-          nbuf ^= 1;
-          prepare(nxt, nxt_first, nbuf);
-        }
         // K of tile j: its slot frees when the score MMA of tile j - NK is done
         const int ks = j % NK;
         if (j >= NK && !wwait(&k_empty[ks], ((j / NK) - 1) & 1)) {
@@ -423,7 +407,86 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         __syncwarp();
       }
       if (!alive) break;
+      if (lane == 0) mbar_arrive(&sched_empty[ss]);  // this item's block ids are no longer needed
       ++k;
+      ++q;
+    }
+  } else if (warp == 10) {
+    // ======================================================== scheduler warp
+    // Takes items (the CTA's first is its own index, later ones come from the tagged
+    // counter), skips empty partitions, reads the context length and the item's
+    // block ids, and queues them for the producer QS deep, so none of these dependent
+    // global reads sit on the TMA producer's path.
+    int q = 0;
+    bool first_take = true;
+    while (true) {
+      const int slot = q % QS;
+      if (q >= QS && !wwait(&sched_empty[slot], ((q / QS) - 1) & 1)) break;
+      ItemDesc d;
+      int first_blk = 0;
+      while (true) {
+        unsigned idx = 0;
+        bool ok = true;
+        if (first_take) {
+          idx = blockIdx.x;
+          first_take = false;
+        } else {
+          if (lane == 0) idx = tagged_fetch_add(p.counters, p.tag, p.err, &ok) + gridDim.x;
+          idx = __shfl_sync(0xffffffffu, idx, 0);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        if (*abort_flag) ok = false;
+        if (!ok || idx >= p.total_items) {
+          d.stop = 1;
+          d.ntiles = 0;
+          break;
+        }
+        const int g = idx % p.num_kv_heads;
+        const unsigned rr = idx / p.num_kv_heads;
+        const int s = rr % p.num_seqs;
+        const int part = rr / p.num_seqs;
+        int ctx = __ldg(p.context_lens + s);
+        if (ctx > p.max_context_len) {
+          if (lane == 0 && part == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+          ctx = p.max_context_len;
+        }
+        if (part * p.partition_size >= ctx) {
+          if (part == 0) {  // empty context: a zero output row
+            for (int i = lane; i < G * HD; i += 32)
+              p.out[(static_cast<int64_t>(s) * Hq + g * G) * HD + i] = __float2bfloat16(0.f);
+          }
+          continue;
+        }
+        const int t0 = part * p.partition_size;
+        const int n = min(ctx - t0, p.partition_size);
+        const int ntiles = (n + TM - 1) / TM;
+        first_blk = t0 >> p.bs_log2;
+        const int nb = ((t0 + ntiles * TM - 1) >> p.bs_log2) - first_blk + 1;
+        int* idb = ids + slot * kMaxIds;
+        for (int i = lane; i < nb && i < kMaxIds; i += 32) {
+          const int b = first_blk + i;
+          int id = b < p.max_blocks
+                       ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b)
+                       : -1;
+          if (id < 0 || id >= p.num_blocks) {
+            if ((b << p.bs_log2) < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+            id = 0;  // in-bounds stand-in; positions past ctx are masked
+          }
+          idb[i] = id;
+        }
+        d.s = s; d.g = g; d.p = part; d.t0 = t0; d.n = n; d.ntiles = ntiles;
+        d.nparts = (ctx + p.partition_size - 1) / p.partition_size;
+        d.stop = 0;
+        break;
+      }
+      __syncwarp();  // the block ids are in shared memory before lane 0 publishes
+      if (lane == 0) {
+        sched_desc[slot] = d;
+        sched_fb[slot] = first_blk;
+        mbar_arrive(&sched_full[slot]);
+      }
+      if (d.stop) break;
+      ++q;
     }
   } else if (warp == 5) {
     // ======================================================== tensor-core issuer
@@ -644,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       if (bar_or(1, 128, failed)) break;
       ++k;
     }
-  } else {
+  } else if (warp < 10) {
     // ======================================================== epilogue warps 6-9
     // warp w reads TMEM lanes 32*(w%4)..+31: thread dl owns output dim dl of the item.
     // Same uniform-exit rule as the softmax group (barrier 2).
@@ -690,11 +753,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             p.ws_ml[pr * 2 + 1] = L[h];
           }
         }
-        __threadfence();
+        // the partial written by all 128 threads, then one release by the leader:
+        // barrier (CTA order) + fence (device scope) + arrival
         named_bar_sync(2, 128);
         if (leader) {
+          __threadfence();
           bool okc = true;
-          const unsigned before = tagged_fetch_add(p.counters + 1 + row0, p.tag, p.err, &okc);
+          const unsigned before = tagged_arrive(p.counters + 1 + row0, p.tag, p.err, &okc);
           *last_flag = okc && (before == static_cast<unsigned>(d.nparts - 1));
           __threadfence();
         }

@@ -39,6 +39,10 @@ constexpr int kOffBar = kOffP + kTileBytes;
 constexpr int kNumBars = 12;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1 KB
+static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
+              "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
+static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 256;               // S: cols 0-127, O: cols 128-255
 
