@@ -197,6 +197,14 @@ class GpuRunner:
         if w.kind == "decode":
             self.ws, self.P = pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads,
                                                   w.head_dim, w.max_context_len, partition_size)
+            # kernels one pa_decode launches: the persistent tcgen05 kernel merges its
+            # partitions itself (head dim 128, partition a multiple of 128 up to 2048);
+            # the CUDA-core kernel adds a reduce launch when the context is split
+            G = w.num_q_heads // w.num_kv_heads
+            tc = (w.head_dim == 128 and G in (1, 2, 4, 8, 16) and self.P % 128 == 0
+                  and self.P <= 2048)
+            split = self.P < w.max_context_len
+            self.decode_launches = 1 if tc or not split else 2
         self.max_q = int(np.max(np.diff(w.cu_seqlens_q))) if w.num_seqs else 0
         torch.cuda.synchronize()
 
@@ -216,7 +224,7 @@ class GpuRunner:
         if w.kind == "decode":
             pa.pa_decode(out, q, self.k_cache, self.v_cache, bt, ctx, w.scale,
                          w.max_context_len, self.P, self.ws)
-            return 2 if self.ws is not None else 1
+            return self.decode_launches
         pa.pa_prefill(out, q, self.k_cache, self.v_cache, bt, self.cu, ctx, w.scale, self.max_q)
         return 1
 

@@ -7,16 +7,22 @@
 // One CTA = 128 query rows of one (sequence, query head). Per KV tile of 128
 // positions:  S = Q K^T  (tcgen05.mma, M=128 N=128 K=128, fp32 in TMEM)
 //             softmax on S, one thread per query row (row max / sum stay in the
-//             thread; no shuffles), P written to shared memory as bf16
-//             O += P V    (tcgen05.mma, accumulator in TMEM, rescaled in place when
-//                          the running max moves)
+//             thread; no shuffles), P written back to TMEM as bf16
+//             O += P V    (tcgen05.mma with A = P read from TMEM, B = V from shared
+//                          memory, accumulator in TMEM)
 // Roles (192 threads): warps 0-3 softmax + epilogue (warp w owns TMEM lanes
-// 32w..32w+31), warp 4 issues TMA loads (Q once, K/V tiles double-buffered and
-// gathered block by block through the block table), warp 5 owns the TMEM
-// allocation and issues the MMAs from one thread. S(j+1) is issued before PV(j),
-// so the tensor core works on the next scores while the softmax runs.
-// Operands use the 128-byte swizzled K-major layout (Q, K, P) and the MN-major
-// layout (V, whose head dim is contiguous), both produced directly by TMA.
+// 32w..32w+31), warp 4 issues TMA loads (Q once; K and V tiles gathered block by
+// block through the block table into two 3-deep rings: a K slot frees when its score
+// MMA is done, a V slot when its value MMA is done), warp 5 owns the TMEM allocation
+// and issues the MMAs from one thread: S(j), then O += P V for tile j-1.
+// S and P are double-buffered in TMEM, and O is rescaled only when a row's running
+// max grows by more than 2^8 (probabilities stay <= 256: in range for bf16). So the
+// softmax of tile j waits neither for the value MMA of tile j-1 (except on a rare
+// rescale) nor for a shared P buffer: its exp2 work overlaps the next score MMA and
+// the previous value MMA. Keeping P in TMEM also keeps it off shared memory, whose
+// bandwidth the score MMA (Q and K both from shared memory) and the TMA writes use.
+// Shared-memory operands use the 128-byte swizzled K-major layout (Q, K) and the
+// MN-major layout (V, whose head dim is contiguous), both produced directly by TMA.
 #include <cuda_bf16.h>
 
 #include "pa_internal.h"
@@ -32,19 +38,23 @@ constexpr int kThreads = 192;
 constexpr int kRegion = BM * 128;  // one 64-column half of a 128x128 bf16 tile (16 KB)
 constexpr int kTileBytes = 2 * kRegion;
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;       // 2 stages
-constexpr int kOffV = kOffK + 2 * kTileBytes;   // 2 stages
-constexpr int kOffP = kOffV + 2 * kTileBytes;
-constexpr int kOffBar = kOffP + kTileBytes;
-constexpr int kNumBars = 12;
+constexpr int NKV = 3;                           // K ring and V ring depth
+constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffV = kOffK + NKV * kTileBytes;
+constexpr int kOffBar = kOffV + NKV * kTileBytes;
+// q, mma drain, k/v full/empty (NKV each), s full/free, p full, pv done (2 each)
+constexpr int kNumBars = 2 + 4 * NKV + 4 * 2;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1 KB
-static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
+static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
               "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kTmemCols = 256;               // S: cols 0-127, O: cols 128-255
+constexpr float kRescaleLog2 = 8.f;   // rescale O only past this growth of the row max
+constexpr uint32_t kTmemCols = 512;   // S[0] 0-127, S[1] 128-255, O 256-383, P[0] 384-447, P[1] 448-511
+constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemP = 384;      // P: 128 bf16 per row = 64 columns
 
 struct PrefillParams {
   __nv_bfloat16* out;
@@ -78,6 +88,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, un
   }
 }
 
+// kPosScale: scale > 0, so the row max can be taken on the raw scores and the scale
+// folded into the exponent's FMA; otherwise (scale <= 0) the scores are scaled first.
+template <bool kPosScale>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -102,35 +115,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     if (tid == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
     return;
   }
-  const int first = ctx - n_new;                       // position of the first new token
+  const int first = ctx - n_new;                          // position of the first new token
   const int rows_valid = min(BM, n_new - qt * BM);
-  const int pos_max = first + qt * BM + rows_valid - 1;  // last visible position in the tile
+  const int pos_max = first + qt * BM + rows_valid - 1;   // last visible position in the tile
   const int ntiles = pos_max / BN + 1;
   const int bs = 1 << p.bs_log2;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* bar_kfull = bars + 1;    // [2]
-  uint64_t* bar_vfull = bars + 3;    // [2]
-  uint64_t* bar_kvempty = bars + 5;  // [2]
-  uint64_t* bar_sfull = bars + 7;
-  uint64_t* bar_sfree = bars + 8;
-  uint64_t* bar_pfull = bars + 9;
-  uint64_t* bar_pvdone = bars + 10;
+  uint64_t* bar_q = bars;
+  uint64_t* mma_drain = bars + 1;
+  uint64_t* k_full = bars + 2;               // [NKV] each
+  uint64_t* k_empty = k_full + NKV;
+  uint64_t* v_full = k_empty + NKV;
+  uint64_t* v_empty = v_full + NKV;
+  uint64_t* s_full = v_empty + NKV;          // [2] each
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_kfull[i], 1);
-      mbar_init(&bar_vfull[i], 1);
-      mbar_init(&bar_kvempty[i], 1);
+    mbar_init(mma_drain, 1);
+    for (int i = 0; i < NKV; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_sfree, BM);
-    mbar_init(bar_pfull, BM);
-    mbar_init(bar_pvdone, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);   // one arrival per softmax warp
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -142,11 +161,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;
-  const uint32_t tO = tmem + 128;
+  const uint32_t tO = tmem + kTmemO;
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
+    // lane 0 waits and issues; the verdict of each wait is broadcast so the warp
+    // leaves the loop together
+    auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
+      int okw = 0;
+      if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, okw, 0) != 0;
+    };
+    const int rows = bs < BN ? bs : BN;
+    const int nbox = BN / rows;
+    const uint64_t keep = policy_evict_last();  // K/V tiles are re-read by G heads and q tiles
+    auto block_row = [&](int pos) {
+      const int bi = pos >> p.bs_log2;
+      int id = bi < p.max_blocks
+                   ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + bi)
+                   : -1;
+      if (id < 0 || id >= p.num_blocks) {
+        if (pos < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+        id = 0;  // in-bounds stand-in; positions past the context are masked
+      }
+      return id * bs + (pos & (bs - 1));
+    };
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
@@ -155,159 +194,201 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       mbar_arrive_expect_tx(bar_q, kTileBytes);
       tma_load_3d(smem + kOffQ, &tmQ, bar_q, 0, h, qrow);
       tma_load_3d(smem + kOffQ + kRegion, &tmQ, bar_q, 64, h, qrow);
-      const int rows = bs < BN ? bs : BN;
-      const int nbox = BN / rows;
-      const uint64_t keep = policy_evict_last();  // K/V tiles are re-read by G heads / q tiles
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !wait_or_abort(&bar_kvempty[st], ((j >> 1) - 1) & 1, p.err, abort_flag))
-          break;
-        uint8_t* kdst = smem + kOffK + st * kTileBytes;
-        uint8_t* vdst = smem + kOffV + st * kTileBytes;
-        mbar_arrive_expect_tx(&bar_kfull[st], kTileBytes);
-        mbar_arrive_expect_tx(&bar_vfull[st], kTileBytes);
-        for (int b = 0; b < nbox; ++b) {
-          const int pos = j * BN + b * rows;
-          const int bi = pos >> p.bs_log2;
-          int id = bi < p.max_blocks
-                       ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + bi)
-                       : -1;
-          if (id < 0 || id >= p.num_blocks) {
-            if (pos < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
-            id = 0;
-          }
-          const int row = id * bs + (pos & (bs - 1));
-          tma_load_3d_hint(kdst + b * rows * 128, &tmK, &bar_kfull[st], 0, g, row, keep);
-          tma_load_3d_hint(kdst + kRegion + b * rows * 128, &tmK, &bar_kfull[st], 64, g, row, keep);
-          tma_load_3d_hint(vdst + b * rows * 128, &tmV, &bar_vfull[st], 0, g, row, keep);
-          tma_load_3d_hint(vdst + kRegion + b * rows * 128, &tmV, &bar_vfull[st], 64, g, row, keep);
+    }
+    int k_issued = 0, v_issued = 0;
+    for (int j = 0; j < ntiles; ++j) {
+      const int b = j % NKV;
+      const unsigned prev = ((j / NKV) - 1) & 1;  // phase of the slot's previous use
+      if (j >= NKV && !wwait(&k_empty[b], prev)) break;
+      if (lane == 0) {
+        uint8_t* dst = smem + kOffK + b * kTileBytes;
+        mbar_arrive_expect_tx(&k_full[b], kTileBytes);
+        for (int c = 0; c < nbox; ++c) {
+          const int row = block_row(j * BN + c * rows);
+          tma_load_3d_hint(dst + c * rows * 128, &tmK, &k_full[b], 0, g, row, keep);
+          tma_load_3d_hint(dst + kRegion + c * rows * 128, &tmK, &k_full[b], 64, g, row, keep);
         }
       }
+      k_issued = j + 1;
+      if (j >= NKV && !wwait(&v_empty[b], prev)) break;
+      if (lane == 0) {
+        uint8_t* dst = smem + kOffV + b * kTileBytes;
+        mbar_arrive_expect_tx(&v_full[b], kTileBytes);
+        for (int c = 0; c < nbox; ++c) {
+          const int row = block_row(j * BN + c * rows);
+          tma_load_3d_hint(dst + c * rows * 128, &tmV, &v_full[b], 0, g, row, keep);
+          tma_load_3d_hint(dst + kRegion + c * rows * 128, &tmV, &v_full[b], 64, g, row, keep);
+        }
+      }
+      v_issued = j + 1;
+    }
+    // Before the CTA ends, every copy this warp started must have landed. Per slot
+    // only the last load can still be in flight (the one before it was consumed),
+    // so waiting for those is enough; on the normal path they completed long ago.
+    if (lane == 0) {
+      mbar_wait(bar_q, 0, p.err);
+      for (int t = k_issued - NKV > 0 ? k_issued - NKV : 0; t < k_issued; ++t)
+        mbar_wait(&k_full[t % NKV], (t / NKV) & 1, p.err);
+      for (int t = v_issued - NKV > 0 ? v_issued - NKV : 0; t < v_issued; ++t)
+        mbar_wait(&v_full[t % NKV], (t / NKV) & 1, p.err);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);  // Q K-major, K K-major
-      constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);  // P K-major, V MN-major
+      constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);  // P (TMEM), V MN-major
       const uint32_t sQ = smem_u32(smem + kOffQ);
-      const uint32_t sP = smem_u32(smem + kOffP);
-      auto pv = [&](int i) -> bool {
-        if (!wait_or_abort(bar_pfull, i & 1, p.err, abort_flag)) return false;
-        if (!wait_or_abort(&bar_vfull[i & 1], (i >> 1) & 1, p.err, abort_flag)) return false;
+      auto pv = [&](int t) -> bool {
+        const int b = t & 1;
+        const int vs = t % NKV;
+        if (!wait_or_abort(&p_full[b], (t >> 1) & 1, p.err, abort_flag) ||
+            !wait_or_abort(&v_full[vs], (t / NKV) & 1, p.err, abort_flag))
+          return false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + kOffV + (i & 1) * kTileBytes);
+        const uint32_t tP = tmem + kTmemP + b * (BN / 2);
+        const uint32_t sV = smem_u32(smem + kOffV + vs * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sP + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
-          tc_mma_f16_ss(tO, a, b, idO, (i > 0 || kk > 0) ? 1u : 0u);
+          // 16 kv positions per step = 8 packed columns of P
+          const uint64_t bd = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
+          tc_mma_f16_ts(tO, tP + kk * 8, bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar_pvdone);
-        tc_commit(&bar_kvempty[i & 1]);
+        tc_commit(&pv_done[b]);
+        tc_commit(&v_empty[vs]);
         return true;
       };
       bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag);
       for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j & 1;
-        if (!wait_or_abort(&bar_kfull[st], (j >> 1) & 1, p.err, abort_flag)) break;
-        if (j > 0 && !wait_or_abort(bar_sfree, (j - 1) & 1, p.err, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t sK = smem_u32(smem + kOffK + st * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(sQ + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(sK + off, 16, 1024);
-          tc_mma_f16_ss(tS, a, b, idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar_sfull);
-        if (j > 0 && !pv(j - 1)) {
+        const int b = j & 1;
+        const int ks = j % NKV;
+        if (!wait_or_abort(&k_full[ks], (j / NKV) & 1, p.err, abort_flag) ||
+            (j >= 2 && !wait_or_abort(&s_free[b], ((j >> 1) - 1) & 1, p.err, abort_flag))) {
           ok = false;
           break;
         }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+          tc_mma_f16_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
+                        smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[b]);
+        tc_commit(&k_empty[ks]);
+        if (j > 0) ok = pv(j - 1);
       }
-      if (ok && !*abort_flag) pv(ntiles - 1);
+      if (ok) pv(ntiles - 1);
+      // every MMA this thread issued has finished before TMEM and shared memory go away
+      tc_commit(mma_drain);
+      mbar_wait(mma_drain, 0, p.err);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
+    // Every lane runs every step (the tcgen05 loads and stores are warp-collective):
+    // a failed wait only marks `failed`, so no lane strands the others.
     const int r = tid;  // query row within the tile == TMEM lane
     const int pos_r = first + qt * BM + (r < rows_valid ? r : rows_valid - 1);
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    uint8_t* sProw = smem + kOffP + r * 128;
-    const int sw = r & 7;
     float m = -INFINITY;
     float l = 0.f;
-    bool ok = true;
+    bool failed = false;
     for (int j = 0; j < ntiles; ++j) {
-      if (!wait_or_abort(bar_sfull, j & 1, p.err, abort_flag)) {
-        ok = false;
-        break;
-      }
+      const int b = j & 1;
+      failed |= !wait_or_abort(&s_full[b], (j >> 1) & 1, p.err, abort_flag);
       tc_fence_after();
       float sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
-        float t[32];
-        tmem_ld32(tS + lane_off + c * 32, t);
+        float t32[32];
+        tmem_ld32(tmem + b * 128 + lane_off + c * 32, t32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = t[i];
+        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = t32[i];
       }
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar_sfree);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
 
       const int kv0 = j * BN;
-      const bool need_mask = kv0 + BN - 1 > pos_r;
-      float mx = -INFINITY;
+      const int lim = pos_r - kv0;  // columns past lim are in this row's future: masked
+      float mx;
+      if constexpr (kPosScale) {
+        if (lim < BN - 1) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        float x = sv[c] * p.scale_log2;
-        if (need_mask && kv0 + c > pos_r) x = -INFINITY;
-        sv[c] = x;
-        mx = fmaxf(mx, x);
+          for (int c = 0; c < BN; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
+        }
+        // row max of the raw scores (the scale is positive), four independent chains
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; c += 8) {
+          a0 = fmax3(a0, sv[c + 0], sv[c + 1]);
+          a1 = fmax3(a1, sv[c + 2], sv[c + 3]);
+          a2 = fmax3(a2, sv[c + 4], sv[c + 5]);
+          a3 = fmax3(a3, sv[c + 6], sv[c + 7]);
+        }
+        mx = fmax3(a0, a1, fmaxf(a2, a3)) * p.scale_log2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) sv[c] = c > lim ? -INFINITY : sv[c] * p.scale_log2;
+        mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, sv[c]);
       }
-      const float m_new = fmaxf(m, mx);  // finite: position 0 is visible in tile 0
-      const float alpha = ex2_approx(m - m_new);
-      float rs = 0.f;
+      // reference max: the first tile's (position 0 is visible to every row), raised
+      // only when a later tile exceeds it by more than 2^8
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m = mx;
+      } else if (mx > m + kRescaleLog2) {
+        alpha = ex2_approx(m - mx);
+        m = mx;
+        rescale = true;
+      }
+      // p = 2^(s * scale_log2 - m), two lanes of fp32 per instruction
+      const float2 sc2 = make_float2(kPosScale ? p.scale_log2 : 1.f, kPosScale ? p.scale_log2 : 1.f);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(sv[c] - m_new);
-        const float p1 = ex2_approx(sv[c + 1] - m_new);
-        rs += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+        const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
+        pk[c >> 1] = pack_bf16x2(e.x, e.y);
       }
+      const float rs = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                       ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
       l = l * alpha + rs;
-      m = m_new;
 
-      if (j > 0) {
-        if (!wait_or_abort(bar_pvdone, (j - 1) & 1, p.err, abort_flag)) {
-          ok = false;
-          break;
-        }
+      // P buffer b was last read by the value MMA of tile j-2
+      if (j >= 2) failed |= !wait_or_abort(&pv_done[b], ((j >> 1) - 1) & 1, p.err, abort_flag);
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O holds the value MMAs up to tile j-1: wait for the last one, then rescale
+        // (rows that do not need it multiply by 1)
+        const int t = j - 1;
+        failed |= !wait_or_abort(&pv_done[t & 1], (t >> 1) & 1, p.err, abort_flag);
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha < 1.f)) {
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            float t[32];
-            tmem_ld32(tO + lane_off + c * 32, t);
-            tc_wait_ld();
+        for (int c = 0; c < HD / 32; ++c) {
+          float o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
+          tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) t[i] *= alpha;
-            tmem_st32(tO + lane_off + c * 32, t);
-          }
-          tc_wait_st();
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO + lane_off + c * 32, o);
         }
       }
       if (j == ntiles - 1 && ctx - kv0 < BN) {
         // rows past the context in the last V tile may hold anything (even NaN);
-        // P is 0 there but 0 * NaN is NaN, so clear them before PV reads the tile
-        if (!wait_or_abort(&bar_vfull[j & 1], (j >> 1) & 1, p.err, abort_flag)) {
-          ok = false;
-          break;
-        }
+        // P is 0 there but 0 * NaN is NaN, so clear them before the value MMA
+        const int vs = j % NKV;
+        failed |= !wait_or_abort(&v_full[vs], (j / NKV) & 1, p.err, abort_flag);
         if (r >= ctx - kv0) {
-          uint8_t* v = smem + kOffV + (j & 1) * kTileBytes + r * 128;
+          uint8_t* v = smem + kOffV + vs * kTileBytes + r * 128;
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -315,40 +396,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
             *reinterpret_cast<uint4*>(v + kRegion + c * 16) = z;
           }
         }
+        fence_proxy_async_smem();
       }
-      // P row -> shared memory, 128-byte swizzle: chunk c of the row goes to c ^ (row & 7)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int region = c >> 3;
-        const int cc = c & 7;
-        uint4 w = make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-        *reinterpret_cast<uint4*>(sProw + region * kRegion + ((cc ^ sw) << 4)) = w;
-      }
-      fence_proxy_async_smem();
+      // P row -> TMEM: 64 columns of packed bf16 pairs (the A-operand layout)
+      const uint32_t tP = tmem + kTmemP + b * (BN / 2) + lane_off;
+      tmem_st32_bits(tP, pk);
+      tmem_st32_bits(tP + 32, pk + 32);
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pfull);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
     }
-    if (ok && wait_or_abort(bar_pvdone, (ntiles - 1) & 1, p.err, abort_flag)) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool store = r < rows_valid;
-      __nv_bfloat16* orow =
-          p.out + (static_cast<int64_t>(q0 + qt * BM + r) * p.num_q_heads + h) * HD;
+    const int t = ntiles - 1;
+    failed |= !wait_or_abort(&pv_done[t & 1], (t >> 1) & 1, p.err, abort_flag);
+    tc_fence_after();
+    const float inv_l = 1.f / l;
+    const bool store = r < rows_valid && !failed;
+    __nv_bfloat16* orow =
+        p.out + (static_cast<int64_t>(q0 + qt * BM + r) * p.num_q_heads + h) * HD;
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float t[32];
-        tmem_ld32(tO + lane_off + c * 32, t);
-        tc_wait_ld();
-        if (store) {
+    for (int c = 0; c < HD / 32; ++c) {
+      float o[32];
+      tmem_ld32(tO + lane_off + c * 32, o);
+      tc_wait_ld();
+      if (store) {
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16x2(t[v4 * 8 + 0] * inv_l, t[v4 * 8 + 1] * inv_l);
-            w.y = pack_bf16x2(t[v4 * 8 + 2] * inv_l, t[v4 * 8 + 3] * inv_l);
-            w.z = pack_bf16x2(t[v4 * 8 + 4] * inv_l, t[v4 * 8 + 5] * inv_l);
-            w.w = pack_bf16x2(t[v4 * 8 + 6] * inv_l, t[v4 * 8 + 7] * inv_l);
-            *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = w;
-          }
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 w;
+          w.x = pack_bf16x2(o[v4 * 8 + 0] * inv_l, o[v4 * 8 + 1] * inv_l);
+          w.y = pack_bf16x2(o[v4 * 8 + 2] * inv_l, o[v4 * 8 + 3] * inv_l);
+          w.z = pack_bf16x2(o[v4 * 8 + 4] * inv_l, o[v4 * 8 + 5] * inv_l);
+          w.w = pack_bf16x2(o[v4 * 8 + 6] * inv_l, o[v4 * 8 + 7] * inv_l);
+          *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = w;
         }
       }
     }
@@ -389,11 +468,17 @@ cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.total_q = a.total_q;
   p.max_q_len = a.max_q_len;
   p.scale_log2 = a.scale * kLog2e;
-  cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(prefill_kernel), kSmemBytes);
+  const bool pos = a.scale > 0.f;
+  const void* fn = pos ? reinterpret_cast<const void*>(prefill_kernel<true>)
+                       : reinterpret_cast<const void*>(prefill_kernel<false>);
+  cudaError_t e = ensure_max_dynamic_smem(fn, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((a.max_q_len + BM - 1) / BM, a.num_q_heads, a.num_seqs);
   if (grid.x == 0 || a.num_seqs == 0) return cudaSuccess;
-  prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  if (pos)
+    prefill_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  else
+    prefill_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
