@@ -6,21 +6,26 @@
 //
 // One CTA = 128 query rows of one (sequence, query head). Per KV tile of 128
 // positions:  S = Q K^T  (tcgen05.mma, M=128 N=128 K=128, fp32 in TMEM)
-//             softmax on S, one thread per query row (row max / sum stay in the
-//             thread; no shuffles), P written back to TMEM as bf16
+//             softmax on S, P written back to TMEM as bf16
 //             O += P V    (tcgen05.mma with A = P read from TMEM, B = V from shared
 //                          memory, accumulator in TMEM)
-// Roles (192 threads): warps 0-3 softmax + epilogue (warp w owns TMEM lanes
-// 32w..32w+31), warp 4 issues TMA loads (Q once; K and V tiles gathered block by
-// block through the block table into two 3-deep rings: a K slot frees when its score
-// MMA is done, a V slot when its value MMA is done), warp 5 owns the TMEM allocation
-// and issues the MMAs from one thread: S(j), then O += P V for tile j-1.
+// Roles (320 threads):
+//   warps 0-7  softmax + epilogue. Warp w reads TMEM lanes 32(w%4).. (its 32 query
+//              rows) and the column half w/4 of each tile, so every row is shared by
+//              two warps on the same SM sub-partition: two warps per scheduler hide
+//              each other's latencies, and each thread keeps 64 scores in registers.
+//              The two halves agree on the row max through shared memory.
+//   warp 8     TMA producer: Q once, then K and V tiles gathered block by block
+//              through the block table into two 3-deep rings (K runs two tiles ahead
+//              of V; a K slot frees when its score MMA is done, a V slot when its
+//              value MMA is done).
+//   warp 9     owns the TMEM allocation and issues the MMAs from one thread.
 // S and P are double-buffered in TMEM, and O is rescaled only when a row's running
-// max grows by more than 2^8 (probabilities stay <= 256: in range for bf16). So the
-// softmax of tile j waits neither for the value MMA of tile j-1 (except on a rare
-// rescale) nor for a shared P buffer: its exp2 work overlaps the next score MMA and
-// the previous value MMA. Keeping P in TMEM also keeps it off shared memory, whose
-// bandwidth the score MMA (Q and K both from shared memory) and the TMA writes use.
+// max grows by more than 2^8 (probabilities stay <= 256: in range for bf16). The
+// tensor core runs its queue in order, so S(j+2) is issued as soon as the softmax has
+// read S(j), ahead of O += P(j) V(j): the next scores never queue behind a value MMA
+// that waited for the softmax, and the exp2 work overlaps both MMAs. P never touches
+// shared memory, whose bandwidth the score MMA and the TMA writes use.
 // Shared-memory operands use the 128-byte swizzled K-major layout (Q, K) and the
 // MN-major layout (V, whose head dim is contiguous), both produced directly by TMA.
 #include <cuda_bf16.h>
@@ -34,21 +39,29 @@ namespace {
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // KV positions per tile
 constexpr int HD = 128;          // head dim
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kIssuerWarp = 9;
+constexpr int kThreads = 320;
+constexpr int NK = 3;            // K ring depth
+constexpr int NV = 3;            // V ring depth
+constexpr int kKAhead = 2;       // K loads run this many tiles ahead of V loads
 constexpr int kRegion = BM * 128;  // one 64-column half of a 128x128 bf16 tile (16 KB)
 constexpr int kTileBytes = 2 * kRegion;
-constexpr int kOffQ = 0;
-constexpr int NKV = 3;                           // K ring and V ring depth
+// Small objects first (8-byte aligned at the start of dynamic shared memory), then
+// the 1024-byte-aligned operand tiles.
+constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 4 * 2;  // q, drain, K/V rings, s/p/pv pairs
+constexpr int kOffXch = 8 * kNumBars;                  // [2 halves][128 rows] fp32
+constexpr int kOffMisc = kOffXch + 2 * BM * 4;         // tmem address, abort flag
+constexpr int kSmallBytes = kOffMisc + 16;
+constexpr int kOffQ = 0;                               // within the aligned region
 constexpr int kOffK = kOffQ + kTileBytes;
-constexpr int kOffV = kOffK + NKV * kTileBytes;
-constexpr int kOffBar = kOffV + NKV * kTileBytes;
-// q, mma drain, k/v full/empty (NKV each), s full/free, p full, pv done (2 each)
-constexpr int kNumBars = 2 + 4 * NKV + 4 * 2;
-constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1 KB
-static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
+constexpr int kOffV = kOffK + NK * kTileBytes;
+constexpr int kDataBytes = kOffV + NV * kTileBytes;
+constexpr int kSmemBytes = kSmallBytes + 1023 + kDataBytes;  // worst-case alignment pad
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0,
               "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
-static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kOffXch % 8 == 0 && kOffMisc % 8 == 0, "mbarriers / words alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;   // rescale O only past this growth of the row max
@@ -88,6 +101,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, un
   }
 }
 
+// named barrier over the two softmax warps that share a group of 32 rows
+__device__ __forceinline__ void pair_sync(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
 // kPosScale: scale > 0, so the row max can be taken on the raw scores and the scale
 // folded into the exponent's FMA; otherwise (scale <= 0) the scores are scaled first.
 template <bool kPosScale>
@@ -95,8 +113,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
+  uint8_t* small = smem_raw;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+      (reinterpret_cast<uintptr_t>(smem_raw + kSmallBytes) + 1023) &
+      ~static_cast<uintptr_t>(1023));
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -121,39 +141,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int ntiles = pos_max / BN + 1;
   const int bs = 1 << p.bs_log2;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(small);
   uint64_t* bar_q = bars;
   uint64_t* mma_drain = bars + 1;
-  uint64_t* k_full = bars + 2;               // [NKV] each
-  uint64_t* k_empty = k_full + NKV;
-  uint64_t* v_full = k_empty + NKV;
-  uint64_t* v_empty = v_full + NKV;
-  uint64_t* s_full = v_empty + NKV;          // [2] each
+  uint64_t* k_full = bars + 2;               // [NK] each
+  uint64_t* k_empty = k_full + NK;
+  uint64_t* v_full = k_empty + NK;           // [NV] each
+  uint64_t* v_empty = v_full + NV;
+  uint64_t* s_full = v_empty + NV;           // [2] each
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+  float* xch = reinterpret_cast<float*>(small + kOffXch);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(small + kOffMisc + 8);
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
     mbar_init(mma_drain, 1);
-    for (int i = 0; i < NKV; ++i) {
+    for (int i = 0; i < NK; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);   // one arrival per softmax warp
-      mbar_init(&p_full[i], 4);
+      mbar_init(&s_free[i], kSoftmaxWarps);   // one arrival per softmax warp
+      mbar_init(&p_full[i], kSoftmaxWarps);
       mbar_init(&pv_done[i], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kIssuerWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -163,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem + kTmemO;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     // lane 0 waits and issues; the verdict of each wait is broadcast so the warp
     // leaves the loop together
@@ -186,6 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       }
       return id * bs + (pos & (bs - 1));
     };
+    auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
+      mbar_arrive_expect_tx(bar, kTileBytes);
+      for (int c = 0; c < nbox; ++c) {
+        const int row = block_row(j * BN + c * rows);
+        tma_load_3d_hint(dst + c * rows * 128, map, bar, 0, g, row, keep);
+        tma_load_3d_hint(dst + kRegion + c * rows * 128, map, bar, 64, g, row, keep);
+      }
+    };
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
@@ -196,53 +227,64 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       tma_load_3d(smem + kOffQ + kRegion, &tmQ, bar_q, 64, h, qrow);
     }
     int k_issued = 0, v_issued = 0;
-    for (int j = 0; j < ntiles; ++j) {
-      const int b = j % NKV;
-      const unsigned prev = ((j / NKV) - 1) & 1;  // phase of the slot's previous use
-      if (j >= NKV && !wwait(&k_empty[b], prev)) break;
-      if (lane == 0) {
-        uint8_t* dst = smem + kOffK + b * kTileBytes;
-        mbar_arrive_expect_tx(&k_full[b], kTileBytes);
-        for (int c = 0; c < nbox; ++c) {
-          const int row = block_row(j * BN + c * rows);
-          tma_load_3d_hint(dst + c * rows * 128, &tmK, &k_full[b], 0, g, row, keep);
-          tma_load_3d_hint(dst + kRegion + c * rows * 128, &tmK, &k_full[b], 64, g, row, keep);
-        }
+    for (int step = 0; step < ntiles + kKAhead; ++step) {
+      const int kj = step;            // K(kj) is needed early: by the score MMA
+      const int vj = step - kKAhead;  // V(vj) only once the softmax of vj is done
+      if (kj < ntiles) {
+        const int ks = kj % NK;
+        if (kj >= NK && !wwait(&k_empty[ks], ((kj / NK) - 1) & 1)) break;
+        if (lane == 0) load_tile(&tmK, smem + kOffK + ks * kTileBytes, &k_full[ks], kj);
+        k_issued = kj + 1;
       }
-      k_issued = j + 1;
-      if (j >= NKV && !wwait(&v_empty[b], prev)) break;
-      if (lane == 0) {
-        uint8_t* dst = smem + kOffV + b * kTileBytes;
-        mbar_arrive_expect_tx(&v_full[b], kTileBytes);
-        for (int c = 0; c < nbox; ++c) {
-          const int row = block_row(j * BN + c * rows);
-          tma_load_3d_hint(dst + c * rows * 128, &tmV, &v_full[b], 0, g, row, keep);
-          tma_load_3d_hint(dst + kRegion + c * rows * 128, &tmV, &v_full[b], 64, g, row, keep);
-        }
+      if (vj >= 0 && vj < ntiles) {
+        const int vs = vj % NV;
+        if (vj >= NV && !wwait(&v_empty[vs], ((vj / NV) - 1) & 1)) break;
+        if (lane == 0) load_tile(&tmV, smem + kOffV + vs * kTileBytes, &v_full[vs], vj);
+        v_issued = vj + 1;
       }
-      v_issued = j + 1;
     }
     // Before the CTA ends, every copy this warp started must have landed. Per slot
     // only the last load can still be in flight (the one before it was consumed),
     // so waiting for those is enough; on the normal path they completed long ago.
     if (lane == 0) {
       mbar_wait(bar_q, 0, p.err);
-      for (int t = k_issued - NKV > 0 ? k_issued - NKV : 0; t < k_issued; ++t)
-        mbar_wait(&k_full[t % NKV], (t / NKV) & 1, p.err);
-      for (int t = v_issued - NKV > 0 ? v_issued - NKV : 0; t < v_issued; ++t)
-        mbar_wait(&v_full[t % NKV], (t / NKV) & 1, p.err);
+      for (int t = k_issued - NK > 0 ? k_issued - NK : 0; t < k_issued; ++t)
+        mbar_wait(&k_full[t % NK], (t / NK) & 1, p.err);
+      for (int t = v_issued - NV > 0 ? v_issued - NV : 0; t < v_issued; ++t)
+        mbar_wait(&v_full[t % NV], (t / NV) & 1, p.err);
     }
-  } else if (warp == 5) {
+  } else if (warp == kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);  // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);  // P (TMEM), V MN-major
       const uint32_t sQ = smem_u32(smem + kOffQ);
+      // S(j) into TMEM buffer j & 1, once K(j) has landed and the softmax has read
+      // S(j-2) out of that buffer
+      auto score = [&](int j) -> bool {
+        const int b = j & 1;
+        const int ks = j % NK;
+        if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag) ||
+            (j >= 2 && !wait_or_abort(&s_free[b], ((j >> 1) - 1) & 1, p.err, abort_flag)))
+          return false;
+        tc_fence_after();
+        const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+          tc_mma_f16_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
+                        smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[b]);
+        tc_commit(&k_empty[ks]);
+        return true;
+      };
+      // O += P(t) V(t), once the softmax has written P(t) and V(t) has landed
       auto pv = [&](int t) -> bool {
         const int b = t & 1;
-        const int vs = t % NKV;
+        const int vs = t % NV;
         if (!wait_or_abort(&p_full[b], (t >> 1) & 1, p.err, abort_flag) ||
-            !wait_or_abort(&v_full[vs], (t / NKV) & 1, p.err, abort_flag))
+            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag))
           return false;
         tc_fence_after();
         const uint32_t tP = tmem + kTmemP + b * (BN / 2);
@@ -258,50 +300,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         return true;
       };
       bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag);
+      if (ok) ok = score(0);
+      if (ok && ntiles > 1) ok = score(1);
       for (int j = 0; ok && j < ntiles; ++j) {
-        const int b = j & 1;
-        const int ks = j % NKV;
-        if (!wait_or_abort(&k_full[ks], (j / NKV) & 1, p.err, abort_flag) ||
-            (j >= 2 && !wait_or_abort(&s_free[b], ((j >> 1) - 1) & 1, p.err, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-          tc_mma_f16_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
-                        smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[b]);
-        tc_commit(&k_empty[ks]);
-        if (j > 0) ok = pv(j - 1);
+        if (j + 2 < ntiles) ok = score(j + 2);
+        if (ok) ok = pv(j);
       }
-      if (ok) pv(ntiles - 1);
       // every MMA this thread issued has finished before TMEM and shared memory go away
       tc_commit(mma_drain);
       mbar_wait(mma_drain, 0, p.err);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // Every lane runs every step (the tcgen05 loads and stores are warp-collective):
-    // a failed wait only marks `failed`, so no lane strands the others.
-    const int r = tid;  // query row within the tile == TMEM lane
+    // Every lane runs every step (the tcgen05 loads and stores are warp-collective,
+    // and the pair barriers count both warps): a failed wait only marks `failed`.
+    constexpr int HC = BN / 2;                // columns per half
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int r = quad * 32 + lane;           // query row within the tile == TMEM lane
     const int pos_r = first + qt * BM + (r < rows_valid ? r : rows_valid - 1);
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int pair_bar = 1 + quad;
+    float* my_x = xch + half * BM + r;
+    const float* other_x = xch + (half ^ 1) * BM + r;
     float m = -INFINITY;
-    float l = 0.f;
+    float l = 0.f;                            // this half's share of the row sum
     bool failed = false;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
       failed |= !wait_or_abort(&s_full[b], (j >> 1) & 1, p.err, abort_flag);
       tc_fence_after();
-      float sv[BN];
+      float sv[HC];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < HC / 32; ++c) {
         float t32[32];
-        tmem_ld32(tmem + b * 128 + lane_off + c * 32, t32);
+        tmem_ld32(tmem + b * 128 + half * HC + lane_off + c * 32, t32);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = t32[i];
       }
@@ -310,33 +343,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
 
-      const int kv0 = j * BN;
+      const int kv0 = j * BN + half * HC;
       const int lim = pos_r - kv0;  // columns past lim are in this row's future: masked
-      float mx;
+      float hmx;
       if constexpr (kPosScale) {
-        if (lim < BN - 1) {
+        if (lim < HC - 1) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
+          for (int c = 0; c < HC; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
         }
-        // row max of the raw scores (the scale is positive), four independent chains
+        // max of the raw scores (the scale is positive), four independent chains
         float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN; c += 8) {
+        for (int c = 0; c < HC; c += 8) {
           a0 = fmax3(a0, sv[c + 0], sv[c + 1]);
           a1 = fmax3(a1, sv[c + 2], sv[c + 3]);
           a2 = fmax3(a2, sv[c + 4], sv[c + 5]);
           a3 = fmax3(a3, sv[c + 6], sv[c + 7]);
         }
-        mx = fmax3(a0, a1, fmaxf(a2, a3)) * p.scale_log2;
+        hmx = fmax3(a0, a1, fmaxf(a2, a3));
       } else {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) sv[c] = c > lim ? -INFINITY : sv[c] * p.scale_log2;
-        mx = -INFINITY;
+        for (int c = 0; c < HC; ++c) sv[c] = c > lim ? -INFINITY : sv[c] * p.scale_log2;
+        hmx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < HC; ++c) hmx = fmaxf(hmx, sv[c]);
       }
+      // the two halves of the row swap their maxima: write, sync, read, sync (the
+      // second sync keeps the next tile's write behind this read)
+      *my_x = hmx;
+      pair_sync(pair_bar);
+      const float omx = *other_x;
+      pair_sync(pair_bar);
+      const float mx = kPosScale ? fmaxf(hmx, omx) * p.scale_log2 : fmaxf(hmx, omx);
       // reference max: the first tile's (position 0 is visible to every row), raised
-      // only when a later tile exceeds it by more than 2^8
+      // only when a later tile exceeds it by more than 2^8; both halves compute the
+      // same value from the same inputs
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -347,13 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         rescale = true;
       }
       // p = 2^(s * scale_log2 - m), two lanes of fp32 per instruction
-      const float2 sc2 = make_float2(kPosScale ? p.scale_log2 : 1.f, kPosScale ? p.scale_log2 : 1.f);
+      const float sc = kPosScale ? p.scale_log2 : 1.f;
+      const float2 sc2 = make_float2(sc, sc);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
-      uint32_t pk[BN / 2];
+      uint32_t pk[HC / 2];
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
+      for (int c = 0; c < HC; c += 2) {
         const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
         acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
@@ -368,40 +410,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       tc_fence_after();
       if (__any_sync(0xffffffffu, rescale)) {
         // O holds the value MMAs up to tile j-1: wait for the last one, then rescale
-        // (rows that do not need it multiply by 1)
+        // this half's columns (rows that do not need it multiply by 1)
         const int t = j - 1;
         failed |= !wait_or_abort(&pv_done[t & 1], (t >> 1) & 1, p.err, abort_flag);
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
+        for (int c = 0; c < HC / 32; ++c) {
           float o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tO + half * HC + lane_off + c * 32, o);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO + lane_off + c * 32, o);
+          tmem_st32(tO + half * HC + lane_off + c * 32, o);
         }
       }
-      if (j == ntiles - 1 && ctx - kv0 < BN) {
+      if (j == ntiles - 1 && ctx - j * BN < BN) {
         // rows past the context in the last V tile may hold anything (even NaN);
-        // P is 0 there but 0 * NaN is NaN, so clear them before the value MMA
-        const int vs = j % NKV;
-        failed |= !wait_or_abort(&v_full[vs], (j / NKV) & 1, p.err, abort_flag);
-        if (r >= ctx - kv0) {
-          uint8_t* v = smem + kOffV + vs * kTileBytes + r * 128;
+        // P is 0 there but 0 * NaN is NaN, so clear them before the value MMA.
+        // Thread (quad, lane, half) clears head-dim half `half` of V row r.
+        const int vs = j % NV;
+        failed |= !wait_or_abort(&v_full[vs], (j / NV) & 1, p.err, abort_flag);
+        if (r >= ctx - j * BN) {
+          uint8_t* v = smem + kOffV + vs * kTileBytes + half * kRegion + r * 128;
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(v + c * 16) = z;
-            *reinterpret_cast<uint4*>(v + kRegion + c * 16) = z;
-          }
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(v + c * 16) = z;
         }
         fence_proxy_async_smem();
       }
-      // P row -> TMEM: 64 columns of packed bf16 pairs (the A-operand layout)
-      const uint32_t tP = tmem + kTmemP + b * (BN / 2) + lane_off;
-      tmem_st32_bits(tP, pk);
-      tmem_st32_bits(tP + 32, pk + 32);
+      // this half of the P row -> TMEM: 32 columns of packed bf16 pairs (the A-operand
+      // layout: row in the lane, consecutive kv positions in consecutive half-words)
+      tmem_st32_bits(tmem + kTmemP + b * (BN / 2) + half * (HC / 2) + lane_off, pk);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -410,14 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int t = ntiles - 1;
     failed |= !wait_or_abort(&pv_done[t & 1], (t >> 1) & 1, p.err, abort_flag);
     tc_fence_after();
-    const float inv_l = 1.f / l;
+    // row sum = both halves' shares (the exchange slots are free: the last read of
+    // them is behind the final pair barrier of the loop)
+    *my_x = l;
+    pair_sync(pair_bar);
+    const float inv_l = 1.f / (l + *other_x);
     const bool store = r < rows_valid && !failed;
     __nv_bfloat16* orow =
-        p.out + (static_cast<int64_t>(q0 + qt * BM + r) * p.num_q_heads + h) * HD;
+        p.out + (static_cast<int64_t>(q0 + qt * BM + r) * p.num_q_heads + h) * HD + half * HC;
 #pragma unroll
-    for (int c = 0; c < HD / 32; ++c) {
+    for (int c = 0; c < HC / 32; ++c) {
       float o[32];
-      tmem_ld32(tO + lane_off + c * 32, o);
+      tmem_ld32(tO + half * HC + lane_off + c * 32, o);
       tc_wait_ld();
       if (store) {
 #pragma unroll
@@ -435,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kIssuerWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
