@@ -10,8 +10,11 @@
 //
 // Grid: one CTA per SM looping over work items (partition p, sequence s, kv head g)
 // taken from a counter in the workspace, so load balances dynamically and the TMA
-// ring never drains between items. Roles (320 threads):
-//   warp 4  producer: takes items, loads q (one box per item) and the K and V tiles
+// ring never drains between items. Roles (352 threads):
+//   warp 10 scheduler: takes the next item from the counter, skips empty partitions
+//           (writing zero rows for empty contexts) and reads the item's block ids, one
+//           item ahead of the producer;
+//   warp 4  producer: loads q (one box per item) and the K and V tiles
 //           of 128 positions through the block table (one TMA box per physical
 //           block) into two 3-deep rings of 32 KB slots. A K slot frees as soon as
 //           its score MMA is done and a V slot when its value MMA is done, so both
