@@ -1,10 +1,12 @@
 #!/usr/bin/env python
 """Benchmark of the B200 paged KV-cache hot path.
 
-Headline workload (one "step"): the decode-batch-64 configuration — store_kvcache
-of the 64 new tokens through the slot mapping, then paged decode attention of the
+Headline workload (one "step"): the decode-batch-64 configuration — the 64 new
+tokens' K/V rows stored through the slot mapping, then paged decode attention of the
 64 sequences (16 q heads / 8 kv heads, head dim 128, block size 256, contexts
-uniform in [512, 4096]) — with the whole pool resident in HBM.
+uniform in [512, 4096]) — with the whole pool resident in HBM. The step is one
+pa_store_decode call (one launch: the decode kernel stores the rows it is about to
+read); --separate-store times pa_store_kvcache + pa_decode instead.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -164,7 +166,7 @@ def prefill_bytes(w):
 
 # --------------------------------------------------------------------------- GPU arm
 class GpuRunner:
-    def __init__(self, w, torch, pa, partition_size=0):
+    def __init__(self, w, torch, pa, partition_size=0, separate_store=False):
         self.w, self.torch, self.pa = w, torch, pa
         dev = torch.device("cuda")
         shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
@@ -205,22 +207,32 @@ class GpuRunner:
                   and self.P <= 2048)
             split = self.P < w.max_context_len
             self.decode_launches = 1 if tc or not split else 2
+        # a decode step that stores new tokens runs as one pa_store_decode call (the
+        # tensor-core kernel stores the rows itself; other shapes add a store launch)
+        self.fused = w.kind == "decode" and self.new_k is not None and not separate_store
+        if self.fused and not tc:
+            self.decode_launches += 1
         self.max_q = int(np.max(np.diff(w.cu_seqlens_q))) if w.num_seqs else 0
         torch.cuda.synchronize()
 
     def store(self, k=None, v=None, slots=None):
-        if self.new_k is None and k is None:
+        if self.fused or (self.new_k is None and k is None):
             return 0
         self.pa.pa_store_kvcache(self.new_k if k is None else k, self.new_v if v is None else v,
                                  self.k_cache, self.v_cache, self.new_slots if slots is None else slots)
         return 1
 
-    def attend(self, q=None, ctx=None, bt=None, out=None):
+    def attend(self, q=None, ctx=None, bt=None, out=None, k=None, v=None, slots=None):
         w, pa = self.w, self.pa
         q = self.q if q is None else q
         out = self.out if out is None else out
         ctx = self.context_lens if ctx is None else ctx
         bt = self.block_tables if bt is None else bt
+        if self.fused:
+            pa.pa_store_decode(self.new_k if k is None else k, self.new_v if v is None else v,
+                               self.new_slots if slots is None else slots, out, q, self.k_cache,
+                               self.v_cache, bt, ctx, w.scale, w.max_context_len, self.P, self.ws)
+            return self.decode_launches
         if w.kind == "decode":
             pa.pa_decode(out, q, self.k_cache, self.v_cache, bt, ctx, w.scale,
                          w.max_context_len, self.P, self.ws)
@@ -293,7 +305,7 @@ def time_e2e(runner, torch, steps, warmup):
             d_k.copy_(h_k, non_blocking=True)
             d_v.copy_(h_v, non_blocking=True)
             runner.store(d_k, d_v, d_slots)
-        runner.attend(d_q, d_ctx, d_bt, d_out)
+        runner.attend(d_q, d_ctx, d_bt, d_out, d_k, d_v, d_slots)
         h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(warmup):
@@ -369,6 +381,8 @@ def main():
                     help="skip the extra per-configuration measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--separate-store", action="store_true",
+                    help="decode steps as pa_store_kvcache + pa_decode instead of pa_store_decode")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -402,7 +416,7 @@ def main():
     hbm_peak, tf_peak, tf_sustained, peak_src = peaks()
     # every rank decodes its own batch of the same shape (weak scaling)
     w = generate(cfg) if rank == 0 else _rank_workload(cfg, rank)
-    runner = GpuRunner(w, torch, pa, args.partition_size)
+    runner = GpuRunner(w, torch, pa, args.partition_size, args.separate_store)
     flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     sampler = ClockSampler(local_rank)
@@ -423,9 +437,13 @@ def main():
     value = world * bytes_step / (step_ms * 1e-3) / 1e9
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
+    if runner.fused:
+        attn_bytes += store_bytes(w)  # the new rows are read and written by the same launch
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     if w.kind == "decode":
-        roofline = {"bound": "hbm", "kernel": "pa_decode (persistent tcgen05 decode, split-K merge fused)",
+        kname = ("pa_store_decode (persistent tcgen05 decode; new-row store and split-K merge inside)"
+                 if runner.fused else "pa_decode (persistent tcgen05 decode, split-K merge inside)")
+        roofline = {"bound": "hbm", "kernel": kname,
                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                     "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
                     "algorithmic_bytes_per_launch": attn_bytes,
@@ -472,7 +490,9 @@ def main():
         "e2e": {"value": round(world * bytes_step / (e2e_step_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_step_ms, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": "paged_kv_cache_442_b200.pa_store_kvcache + pa_decode (C ABI) on pinned host buffers"},
+                "api": ("paged_kv_cache_442_b200.pa_store_decode" if runner.fused else
+                        "paged_kv_cache_442_b200.pa_store_kvcache + pa_decode") +
+                       " (C ABI) on pinned host buffers"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -508,8 +528,8 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
         a_ms = sum(attn_ms) / len(attn_ms)
         d = {"attn_us": round(a_ms * 1e3, 2), "step_us": round(total_ms / n * 1e3, 2), "steps": n}
         if w.kind == "decode":
-            lb = decode_bytes(w)
-            d.update({"kernel": "pa_decode", "logical_bytes": lb, "logical_GBps": round(lb / a_ms / 1e6, 1),
+            lb = decode_bytes(w) + (store_bytes(w) if r.fused else 0)
+            d.update({"kernel": "pa_store_decode" if r.fused else "pa_decode", "logical_bytes": lb, "logical_GBps": round(lb / a_ms / 1e6, 1),
                       "frac_of_hbm_peak_logical": round(lb / a_ms / 1e6 / hbm_peak, 3),
                       "partition_size": r.P})
             if name == "prefix_share_decode":

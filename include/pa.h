@@ -94,8 +94,9 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
 /*
  * Decode split size. The context of every sequence is cut into partitions of
  * partition_size positions (a multiple of 64); each (sequence, kv head,
- * partition) is processed independently and partials are merged by a second
- * kernel. pa_decode_default_partition returns the size pa_decode picks when
+ * partition) is processed independently and the partials are merged at the end
+ * (inside the persistent kernel on the tensor-core path, by a second kernel on
+ * the CUDA-core path). pa_decode_default_partition returns the size pa_decode picks when
  * given partition_size = 0 (depends on the batch, heads, max context and the
  * device's SM count of the current device).
  */
@@ -143,6 +144,38 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int32_t num_q_heads, float scale, int32_t max_context_len,
                     int32_t partition_size, void* workspace, size_t workspace_bytes,
                     void* stream);
+
+/*
+ * pa_store_decode — one decode step of a layer in one call: store this step's
+ * new K/V row of every sequence, then attend (nano vllm page, section 3.1: the
+ * new token's slot is the next position of the sequence's last block; mini-vllm
+ * page, section 2: K/V are written where the block table points, then read
+ * through it). The result, and the pool afterwards, equal pa_store_kvcache
+ * followed by pa_decode with the same arguments.
+ *
+ *   new_k, new_v   [num_seqs, Hkv, D] bf16: the new token's K and V rows.
+ *   slot_mapping   int32 [num_seqs]: -1 = store nothing for that sequence, else
+ *                  the slot of position context_lens[s] - 1 of sequence s
+ *                  (block_tables[s][(ctx-1) / bs] * bs + (ctx-1) % bs). Any other
+ *                  value is not stored and is reported as PA_ERR_BAD_INDEX (debug
+ *                  checks / pa_check_device_errors): the row is written by the
+ *                  part of the kernel that reads that position, just before it
+ *                  reads it, so a slot elsewhere could be read before it is written.
+ *                  The slot must not be read by another sequence of the same call
+ *                  (a block shared by several sequences is copied before it is
+ *                  appended to).
+ *   other arguments as pa_decode.
+ * On the tensor-core path (head dim 128, partition size a multiple of 128 up to
+ * 2048) the store happens inside the decode kernel: one launch per step. Other
+ * shapes launch a checked store kernel and then the decode kernels.
+ */
+pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* slot_mapping,
+                          void* out, const void* q, void* k_cache, void* v_cache,
+                          pa_cache_desc cache, const int32_t* block_tables,
+                          int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_q_heads, float scale,
+                          int32_t max_context_len, int32_t partition_size, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /*
  * pa_decode_no_alloc — pa_decode for callers that cannot allocate device memory.

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
 
 # every extern "C" function include/pa.h declares
 EXPORTED = ("pa_store_kvcache", "pa_decode_default_partition", "pa_decode_workspace_size",
-            "pa_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
+            "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
             "pa_check_device_errors", "pa_status_string", "pa_version")
 
 # size of the library-owned scratch of pa_decode_no_alloc (include/pa.h)
@@ -61,6 +61,9 @@ def load_library(path: str | None = None):
     lib.pa_decode.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32, ctypes.c_float,
                               i32, i32, vp, sz, vp]
     lib.pa_decode.restype = ctypes.c_int
+    lib.pa_store_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
+                                    ctypes.c_float, i32, i32, vp, sz, vp]
+    lib.pa_store_decode.restype = ctypes.c_int
     lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
                                        ctypes.c_float, i32, i32, vp]
     lib.pa_decode_no_alloc.restype = ctypes.c_int
@@ -176,6 +179,42 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                        _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
                        _stream(stream))
     _raise("pa_decode", st)
+
+
+def pa_store_decode(new_k, new_v, slot_mapping, out, q, k_cache, v_cache, block_tables,
+                    context_lens, scale: float, max_context_len: int, partition_size: int = 0,
+                    workspace=None, stream=None) -> None:
+    """Store each sequence's new K/V row at slot_mapping[s] (the slot of its last
+    position, or -1), then decode: the same result as pa_store_kvcache followed by
+    pa_decode, in one launch on the tensor-core path."""
+    torch = _torch()
+    lib = load_library()
+    _check(new_k, "new_k", torch.bfloat16, 3)
+    _check(new_v, "new_v", torch.bfloat16, 3)
+    _check(slot_mapping, "slot_mapping", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    if tuple(out.shape) != (B, Hq, D) or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("out/q/block_tables/context_lens disagree on num_seqs")
+    row = (B, k_cache.shape[2], k_cache.shape[3])
+    if tuple(new_k.shape) != row or tuple(new_v.shape) != row or slot_mapping.shape[0] != B:
+        raise ValueError("new_k/new_v must be [num_seqs, Hkv, D] and slot_mapping [num_seqs]")
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_store_decode(_ptr(new_k), _ptr(new_v), _ptr(slot_mapping), _ptr(out), _ptr(q),
+                             _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
+                             int(block_tables.shape[1]), _ptr(context_lens), int(B), int(Hq),
+                             float(scale), int(max_context_len), int(partition_size),
+                             _ptr(workspace) if workspace is not None else ctypes.c_void_p(0),
+                             ws_bytes, _stream(stream))
+    _raise("pa_store_decode", st)
 
 
 def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,

@@ -121,6 +121,13 @@ struct TcParams {
   int max_context_len;
   unsigned total_items;
   float scale_log2;
+  // fused store (pa_store_decode), else all NULL: row s of new_k / new_v goes to the
+  // slot slot_mapping[s], which must be the slot of the sequence's last position
+  const uint4* new_k;        // [B, Hkv, D] bf16, 16 vectors per head
+  const uint4* new_v;
+  const int32_t* slot_mapping;
+  uint4* k_rows;             // the pools, as rows of Hkv x 16 vectors
+  uint4* v_rows;
 };
 
 struct ItemDesc {
@@ -363,6 +370,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         break;
       }
       const int g = cur.g, t0 = cur.t0, ntiles = cur.ntiles;
+      if (p.slot_mapping != nullptr && cur.p == cur.nparts - 1) {
+        // pa_store_decode: this item reads the sequence's last position, so it writes
+        // that position's new row for its kv head first (lanes 0-15: the 16 vectors
+        // of K, lanes 16-31: V), then makes the writes visible to its TMA loads.
+        // Only the slot the block table gives for that position is accepted.
+        const int pos = t0 + cur.n - 1;
+        const int bi = (pos >> p.bs_log2) - first_blk;
+        const int64_t expect =
+            static_cast<int64_t>(bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+        const int dst_slot = __ldg(p.slot_mapping + cur.s);
+        if (dst_slot >= 0) {
+          if (dst_slot != expect) {
+            if (lane == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+          } else {
+            const int64_t src = (static_cast<int64_t>(cur.s) * p.num_kv_heads + g) * 16 + (lane & 15);
+            const int64_t dst = (static_cast<int64_t>(dst_slot) * p.num_kv_heads + g) * 16 + (lane & 15);
+            if (lane < 16)
+              p.k_rows[dst] = __ldg(p.new_k + src);
+            else
+              p.v_rows[dst] = __ldg(p.new_v + src);
+            fence_proxy_async_global();
+          }
+        }
+        __syncwarp();
+      }
       if (lane == 0) {
         descs[slot] = cur;
         mbar_arrive_expect_tx(&item_full[slot], 2 * G * 128);
@@ -457,6 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           if (part == 0) {  // empty context: a zero output row
             for (int i = lane; i < G * HD; i += 32)
               p.out[(static_cast<int64_t>(s) * Hq + g * G) * HD + i] = __float2bfloat16(0.f);
+            // and no last position to store a new row at
+            if (p.slot_mapping != nullptr && lane == 0 && __ldg(p.slot_mapping + s) >= 0)
+              flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
           }
           continue;
         }
@@ -860,6 +895,11 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
   p.max_context_len = a.max_context_len;
   p.total_items = static_cast<unsigned>(a.max_parts) * a.num_seqs * a.cache.num_kv_heads;
   p.scale_log2 = a.scale * kLog2e;
+  p.new_k = static_cast<const uint4*>(a.new_k);
+  p.new_v = static_cast<const uint4*>(a.new_v);
+  p.slot_mapping = a.slot_mapping;
+  p.k_rows = static_cast<uint4*>(const_cast<void*>(a.k_cache));
+  p.v_rows = static_cast<uint4*>(const_cast<void*>(a.v_cache));
   switch (a.num_q_heads / a.cache.num_kv_heads) {
     case 1: return launch_tc_t<1>(a, p, stream);
     case 2: return launch_tc_t<2>(a, p, stream);

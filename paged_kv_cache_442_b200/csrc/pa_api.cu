@@ -125,6 +125,93 @@ bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uin
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
+// pa_decode, and pa_store_decode when `store` carries the new rows and slots
+struct StoreRows {
+  const void* new_k;
+  const void* new_v;
+  const int32_t* slot_mapping;
+};
+
+pa_status decode_impl(const StoreRows* store, void* out, const void* q, const void* k_cache,
+                      const void* v_cache, pa_cache_desc cache, const int32_t* block_tables,
+                      int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
+                      int32_t num_q_heads, float scale, int32_t max_context_len,
+                      int32_t partition_size, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache.num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) >
+      static_cast<int64_t>(max_blocks_per_seq) * cache.block_size)
+    return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache.num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && !(G == 16 && cache.head_dim == 128))
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (store && (!store->new_k || !store->new_v || !store->slot_mapping ||
+                !aligned16(store->new_k) || !aligned16(store->new_v)))
+    return PA_ERR_INVALID_ARG;
+  if (partition_size < 0 || (partition_size % 64) != 0) return PA_ERR_INVALID_ARG;
+  const int P = partition_size > 0 ? partition_size
+                                   : pa_decode_default_partition(num_seqs, cache.num_kv_heads,
+                                                                 max_context_len);
+  const int64_t parts64 = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
+  // work items are counted in 24 bits, with room for one extra take per CTA
+  if (parts64 * num_seqs * cache.num_kv_heads >= (1ll << 24) - 4096) return PA_ERR_UNSUPPORTED;
+  const int parts = static_cast<int>(parts64);
+  const size_t need =
+      pa_decode_workspace_size(num_seqs, num_q_heads, cache.head_dim, max_context_len, P);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+
+  DecodeLaunch a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cache = cache;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.scale = scale;
+  a.max_context_len = max_context_len;
+  a.partition_size = P;
+  a.max_parts = parts;
+  const size_t cbytes = decode_counter_bytes(num_seqs, num_q_heads);
+  unsigned long long* counters = static_cast<unsigned long long*>(workspace);
+  float* ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
+  a.ws_o = parts > 1 ? ws : nullptr;
+  a.ws_ml = parts > 1 ? ws + static_cast<size_t>(num_seqs) * num_q_heads * parts * cache.head_dim
+                      : nullptr;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (store) {
+    a.new_k = store->new_k;
+    a.new_v = store->new_v;
+    a.slot_mapping = store->slot_mapping;
+  }
+  // the persistent kernel stores the new rows itself; the CUDA-core path stores them
+  // with a checked kernel first
+  if (decode_tc_supported(a)) return finish(launch_decode_tc(a, counters, s), stream);
+  if (G == 16) return PA_ERR_UNSUPPORTED;
+  if (store) {
+    const cudaError_t e = launch_store_last_rows(a, s);
+    if (e != cudaSuccess) return finish(e, stream);
+  }
+  return finish(launch_decode(a, s), stream);
+}
+
+}  // namespace
+
 }  // namespace pa
 
 using namespace pa;
@@ -209,65 +296,28 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
          static_cast<size_t>(num_seqs) * num_q_heads * parts * (head_dim + 2) * sizeof(float);
 }
 
+
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     pa_cache_desc cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
                     const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
                     float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
                     size_t workspace_bytes, void* stream) {
-  pa_status st = check_cache(cache);
-  if (st != PA_OK) return st;
-  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
-    return PA_ERR_INVALID_ARG;
-  if (num_q_heads % cache.num_kv_heads) return PA_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(max_context_len) >
-      static_cast<int64_t>(max_blocks_per_seq) * cache.block_size)
-    return PA_ERR_INVALID_ARG;
-  const int G = num_q_heads / cache.num_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8 && !(G == 16 && cache.head_dim == 128))
-    return PA_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
-    return PA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return PA_ERR_INVALID_ARG;
-  if (partition_size < 0 || (partition_size % 64) != 0) return PA_ERR_INVALID_ARG;
-  const int P = partition_size > 0 ? partition_size
-                                   : pa_decode_default_partition(num_seqs, cache.num_kv_heads,
-                                                                 max_context_len);
-  const int64_t parts64 = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
-  // work items are counted in 24 bits, with room for one extra take per CTA
-  if (parts64 * num_seqs * cache.num_kv_heads >= (1ll << 24) - 4096) return PA_ERR_UNSUPPORTED;
-  const int parts = static_cast<int>(parts64);
-  const size_t need =
-      pa_decode_workspace_size(num_seqs, num_q_heads, cache.head_dim, max_context_len, P);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+  return decode_impl(nullptr, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                     context_lens, num_seqs, num_q_heads, scale, max_context_len, partition_size,
+                     workspace, workspace_bytes, stream);
+}
 
-  DecodeLaunch a;
-  a.out = out;
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.cache = cache;
-  a.block_tables = block_tables;
-  a.max_blocks_per_seq = max_blocks_per_seq;
-  a.context_lens = context_lens;
-  a.num_seqs = num_seqs;
-  a.num_q_heads = num_q_heads;
-  a.scale = scale;
-  a.max_context_len = max_context_len;
-  a.partition_size = P;
-  a.max_parts = parts;
-  const size_t cbytes = decode_counter_bytes(num_seqs, num_q_heads);
-  unsigned long long* counters = static_cast<unsigned long long*>(workspace);
-  float* ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
-  a.ws_o = parts > 1 ? ws : nullptr;
-  a.ws_ml = parts > 1 ? ws + static_cast<size_t>(num_seqs) * num_q_heads * parts * cache.head_dim
-                      : nullptr;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (decode_tc_supported(a)) return finish(launch_decode_tc(a, counters, s), stream);
-  if (G == 16) return PA_ERR_UNSUPPORTED;
-  return finish(launch_decode(a, s), stream);
+pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* slot_mapping,
+                          void* out, const void* q, void* k_cache, void* v_cache,
+                          pa_cache_desc cache, const int32_t* block_tables,
+                          int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_q_heads, float scale,
+                          int32_t max_context_len, int32_t partition_size, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  const StoreRows rows{new_k, new_v, slot_mapping};
+  return decode_impl(&rows, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                     context_lens, num_seqs, num_q_heads, scale, max_context_len, partition_size,
+                     workspace, workspace_bytes, stream);
 }
 
 pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -51,8 +51,16 @@ struct DecodeLaunch {
   int32_t max_parts;       // ceil(max_context_len / partition_size)
   float* ws_o;             // [B, Hq, max_parts, D] fp32 (NULL when max_parts == 1)
   float* ws_ml;            // [B, Hq, max_parts, 2] fp32
+  // pa_store_decode: new rows [B, Hkv, D] stored to slot_mapping[s] (the slot of
+  // position context_lens[s] - 1, or -1) before they are read; all NULL for pa_decode
+  const void* new_k = nullptr;
+  const void* new_v = nullptr;
+  const int32_t* slot_mapping = nullptr;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+// Stores the new rows of a pa_store_decode call on its own (the paths whose decode
+// kernel does not store them): checks each slot against the sequence's last position.
+cudaError_t launch_store_last_rows(const DecodeLaunch& a, cudaStream_t stream);
 
 // Persistent tcgen05 decode (head dim 128). `counters` is the workspace's counter
 // region: 1 + num_seqs * num_q_heads epoch-tagged 64-bit counters.

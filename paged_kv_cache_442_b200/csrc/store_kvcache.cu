@@ -35,7 +35,53 @@ __global__ void __launch_bounds__(256) store_kvcache_kernel(
   }
 }
 
+// The new row of each sequence of a pa_store_decode call, written only when its slot
+// is the slot of the sequence's last position (context_lens[s] - 1) as the block
+// table gives it; any other slot is reported and skipped. One CTA per sequence, one
+// 16-byte vector of K and one of V per thread.
+__global__ void __launch_bounds__(128) store_last_rows_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int32_t* __restrict__ slot_mapping,
+    const int32_t* __restrict__ block_tables, const int32_t* __restrict__ context_lens,
+    int32_t max_blocks, int32_t max_context_len, int32_t bs_log2, int32_t num_blocks,
+    int32_t row_vecs, unsigned* err) {
+  const int s = blockIdx.x;
+  const int slot = __ldg(slot_mapping + s);
+  if (slot < 0) return;
+  const int ctx = __ldg(context_lens + s);
+  const int pos = ctx - 1;
+  bool ok = ctx > 0 && ctx <= max_context_len && (pos >> bs_log2) < max_blocks;
+  int id = -1;
+  if (ok) id = __ldg(block_tables + static_cast<int64_t>(s) * max_blocks + (pos >> bs_log2));
+  ok = ok && id >= 0 && id < num_blocks &&
+       static_cast<int64_t>(slot) ==
+           (static_cast<int64_t>(id) << bs_log2) + (pos & ((1 << bs_log2) - 1));
+  if (!ok) {
+    if (threadIdx.x == 0) flag_error(err, PA_DEV_ERR_BAD_INDEX);
+    return;
+  }
+  for (int c = threadIdx.x; c < row_vecs; c += blockDim.x) {
+    const int64_t src = static_cast<int64_t>(s) * row_vecs + c;
+    const int64_t dst = static_cast<int64_t>(slot) * row_vecs + c;
+    k_cache[dst] = __ldg(k + src);
+    v_cache[dst] = __ldg(v + src);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_store_last_rows(const DecodeLaunch& a, cudaStream_t stream) {
+  if (a.num_seqs == 0 || !a.slot_mapping) return cudaSuccess;
+  const int32_t row_vecs = a.cache.num_kv_heads * a.cache.head_dim * 2 / 16;
+  store_last_rows_kernel<<<a.num_seqs, 128, 0, stream>>>(
+      static_cast<const uint4*>(a.new_k), static_cast<const uint4*>(a.new_v),
+      static_cast<uint4*>(const_cast<void*>(a.k_cache)),
+      static_cast<uint4*>(const_cast<void*>(a.v_cache)), a.slot_mapping, a.block_tables,
+      a.context_lens, a.max_blocks_per_seq, a.max_context_len,
+      31 - __builtin_clz(static_cast<unsigned>(a.cache.block_size)), a.cache.num_blocks, row_vecs,
+      device_error_word());
+  return cudaGetLastError();
+}
 
 cudaError_t launch_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
                                  const pa_cache_desc& c, const int32_t* slot_mapping,

@@ -123,3 +123,31 @@ def test_missing_library_fails_loudly(tmp_path):
             pa.load_library(str(tmp_path / "nope.so"))
     finally:
         pa._lib = saved
+
+
+def test_store_decode_argument_checks(lib):
+    d = desc(hkv=2)
+    ws = FAKE
+    # the new rows are required (and 16-byte aligned) when there are sequences
+    assert lib.pa_store_decode(NULL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1,
+                               32, 0, ws, 1 << 20, NULL) == 1
+    assert lib.pa_store_decode(FAKE, FAKE, NULL, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1,
+                               32, 0, ws, 1 << 20, NULL) == 1
+    misaligned = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.pa_store_decode(misaligned, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4,
+                               0.1, 32, 0, ws, 1 << 20, NULL) == 1
+    # the decode checks still apply: Hq not a multiple of Hkv
+    assert lib.pa_store_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 3, 0.1,
+                               32, 0, ws, 1 << 20, NULL) == 1
+    # empty batch is a no-op
+    assert lib.pa_store_decode(NULL, NULL, NULL, NULL, NULL, NULL, NULL, d, NULL, 4, NULL, 0, 4, 0.1,
+                               32, 0, NULL, 0, NULL) == 0
+
+
+def test_binding_store_decode_shapes():
+    import torch
+    k = torch.zeros(4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_store_decode(k, k, torch.zeros(4, dtype=torch.int32), k, k, k, k,
+                           torch.zeros(4, 4, dtype=torch.int32), torch.zeros(4, dtype=torch.int32),
+                           0.1, 32)
