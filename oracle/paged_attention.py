@@ -71,6 +71,38 @@ def store_kvcache(k_cache: np.ndarray, v_cache: np.ndarray, k: np.ndarray, v: np
 
 
 # ---------------------------------------------------------------------------
+# copy-on-write: a private copy of a shared block before a sequence appends to it
+# ---------------------------------------------------------------------------
+def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, src_blocks: np.ndarray,
+                dst_blocks: np.ndarray):
+    """Return copies of the pools in which block dst_blocks[i] holds what block
+    src_blocks[i] held, in K and in V.
+
+    Blocks are shared between sequences by reference count (nano vllm page, section
+    3.2.1); the page does not say what happens when a sequence writes into a shared
+    block. Reading taken: the writer first gets a private copy (copy-on-write), so
+    the other sharers keep reading the unchanged block. Every source is read before
+    any destination is written; destinations must be distinct and must not also be
+    sources of the same call.
+    """
+    kc = np.array(k_cache, dtype=np.uint16, copy=True)
+    vc = np.array(v_cache, dtype=np.uint16, copy=True)
+    src = [int(b) for b in src_blocks]
+    dst = [int(b) for b in dst_blocks]
+    nb = kc.shape[0]
+    if len(src) != len(dst):
+        raise ValueError("src_blocks and dst_blocks differ in length")
+    if any(b < 0 or b >= nb for b in src + dst):
+        raise IndexError("block id outside the pool")
+    if len(set(dst)) != len(dst) or set(dst) & set(src):
+        raise ValueError("destinations must be distinct and not also sources")
+    for a, b in zip(src, dst):
+        kc[b] = k_cache[a]
+        vc[b] = v_cache[a]
+    return kc, vc
+
+
+# ---------------------------------------------------------------------------
 # a2: logical position -> pool row, and the gather of one sequence
 # ---------------------------------------------------------------------------
 def physical_row(block_table_row: np.ndarray, pos: int, block_size: int) -> int:

@@ -29,6 +29,9 @@ MUTANTS = {
     "store ignores skip": ("        if slot < 0:\n            continue\n", ""),
     "no max subtraction": ("z = z - z.max()", "z = z - z.min()"),
     "prefill scale dropped": ("Z = scale * (qf", "Z = (qf"),
+    "copy direction": ("        kc[b] = k_cache[a]\n        vc[b] = v_cache[a]",
+                       "        kc[a] = k_cache[b]\n        vc[a] = v_cache[b]"),
+    "copy only K": ("        vc[b] = v_cache[a]\n", ""),
 }
 
 
@@ -101,6 +104,14 @@ def _pins(m):
     check("peaked", peaked)
     check("store exact", store_exact)
     check("two-key closed form", two_key_closed_form)
+
+    def cow_append():
+        from tests.test_oracle_pins import cow_workload, run_cow_decode
+        _, (w2, src, dst) = cow_workload(seed=311)
+        out, _ = run_cow_decode(w2, src, dst, m)
+        return np.max(np.abs(out - brute_decode(w2))) < 1e-12
+
+    check("copy-on-write append", cow_append)
     return failed
 
 

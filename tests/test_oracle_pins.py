@@ -269,3 +269,62 @@ def test_compare_reports_both_norms():
     r = np.array([[1.0, 0.0], [0.0, 1.0]])
     c = oracle.compare(r + np.array([[0.0, 0.1], [0.0, 0.0]]), r)
     assert math.isclose(c["max_abs"], 0.1) and math.isclose(c["norm_rel"], 0.1 / math.sqrt(2))
+
+
+# ---------------------------------------------------------------- copy-on-write
+def test_copy_blocks_copies_exactly_the_pairs():
+    rng = np.random.default_rng(51)
+    kc = rng.integers(0, 1 << 16, size=(9, 4, 2, 8), dtype=np.uint16)
+    vc = rng.integers(0, 1 << 16, size=(9, 4, 2, 8), dtype=np.uint16)
+    src, dst = np.array([3, 0, 7]), np.array([5, 8, 1])
+    k2, v2 = oracle.copy_blocks(kc, vc, src, dst)
+    for b in range(9):
+        i = np.where(dst == b)[0]
+        want_k = kc[src[i[0]]] if len(i) else kc[b]
+        want_v = vc[src[i[0]]] if len(i) else vc[b]
+        assert np.array_equal(k2[b], want_k) and np.array_equal(v2[b], want_v)
+    assert np.array_equal(kc[5], kc[5])             # inputs are not modified
+    with pytest.raises(ValueError):
+        oracle.copy_blocks(kc, vc, np.array([1, 2]), np.array([4, 4]))     # duplicate destination
+    with pytest.raises(ValueError):
+        oracle.copy_blocks(kc, vc, np.array([1, 2]), np.array([2, 3]))     # destination is a source
+    with pytest.raises(IndexError):
+        oracle.copy_blocks(kc, vc, np.array([9]), np.array([1]))
+
+
+def cow_workload(seed=61, bs=4):
+    from workloads import copy_on_write_append
+    lens = np.array([3, 20, 14, 17, 40, 8, 16, 6])
+    w = build_workload(kind="decode", context_lens=lens, new_lens=np.zeros_like(lens), num_q_heads=4,
+                       num_kv_heads=2, head_dim=8, block_size=bs, seed=seed, shared_prefix_len=16)
+    return w, copy_on_write_append(w)
+
+
+def run_cow_decode(w2, src, dst, oracle_mod=oracle):
+    """Pools as the sequences left them, shared blocks copied, last rows appended, decode."""
+    kc, vc = w2.empty_pool(), w2.empty_pool()
+    kc, vc = oracle_mod.store_kvcache(kc, vc, w2.setup_k, w2.setup_v, w2.setup_slots)
+    kc, vc = oracle_mod.copy_blocks(kc, vc, src, dst)
+    kc, vc = oracle_mod.store_kvcache(kc, vc, w2.new_k, w2.new_v, w2.new_slots)
+    return oracle_mod.decode(w2.q, kc, vc, w2.block_tables, w2.context_lens, w2.scale), (kc, vc)
+
+
+def test_copy_on_write_append_equals_brute_force_and_keeps_sharers_intact():
+    w, (w2, src, dst) = cow_workload()
+    assert len(src) > 0                                # some last positions were in shared blocks
+    out, (kc, vc) = run_cow_decode(w2, src, dst)
+    assert np.max(np.abs(out - brute_decode(w2))) < TOL
+    # no block is read by one sequence and written in the step by another
+    bs = w2.block_size
+    written = {int(s) // bs for s in w2.new_slots}
+    for s in range(w2.num_seqs):
+        ctx = int(w2.context_lens[s])
+        mine = int(w2.new_slots[np.where(np.nonzero(w2.new_lens)[0] == s)[0][0]]) // bs
+        for b in w2.block_tables[s, :-(-ctx // bs)]:
+            assert int(b) not in written or int(b) == mine
+    # appending without the copies would put rows in blocks other sequences read
+    shared_slots = []
+    for s in range(w.num_seqs):
+        last = int(w.context_lens[s]) - 1
+        shared_slots.append(int(w.block_tables[s, last // bs]) * bs + last % bs)
+    assert len(set(np.array(shared_slots) // bs)) < len(shared_slots)

@@ -289,6 +289,53 @@ def generate(cfg: WorkloadConfig, *, q_factor: float = 1.0, share_prefix: bool =
                           share_prefix=share_prefix, q_factor=q_factor, name=cfg.name)
 
 
+def copy_on_write_append(w: Workload):
+    """A decode step in which every sequence appends (stores) its last position into a
+    block no other sequence of the batch reads.
+
+    With shared prefixes the last position of a short sequence can fall in a block
+    other sequences also read (reference count > 1; nano vllm page, section 3.2.1).
+    Such a block is first copied to a fresh physical block that only this sequence's
+    table points at; the last sharer to append keeps the original. New blocks are
+    appended to the pool (ids num_blocks, num_blocks + 1, ...). This is host-side
+    block management: which blocks to copy, and the resulting tables and slots.
+
+    Returns (workload whose step stores the last row of every sequence,
+             src_blocks int32 [n], dst_blocks int32 [n]).
+    """
+    bs = w.block_size
+    refs = np.zeros(w.num_blocks, dtype=np.int64)
+    for s in range(w.num_seqs):
+        n = -(-int(w.context_lens[s]) // bs)
+        for b in w.block_tables[s, :n]:
+            refs[int(b)] += 1
+    bt = w.block_tables.copy()
+    src, dst, new_slots, new_src = [], [], [], []
+    nxt = w.num_blocks
+    for s in range(w.num_seqs):
+        ctx = int(w.context_lens[s])
+        if ctx <= 0:
+            continue
+        last = ctx - 1
+        bi = last // bs
+        b = int(bt[s, bi])
+        if refs[b] > 1:
+            src.append(b)
+            dst.append(nxt)
+            refs[b] -= 1
+            bt[s, bi] = nxt
+            nxt += 1
+        new_slots.append(int(bt[s, bi]) * bs + last % bs)
+        new_src.append(int(w.logical_rows[s][last]))
+    rc = np.concatenate([refs, np.ones(nxt - w.num_blocks, dtype=np.int64)]).astype(np.int32)
+    w2 = Workload(**{**w.__dict__, "num_blocks": nxt, "block_tables": bt,
+                     "new_lens": (w.context_lens > 0).astype(np.int32),
+                     "new_slots": np.asarray(new_slots, dtype=np.int32),
+                     "new_src": np.asarray(new_src, dtype=np.int64), "ref_counts": rc,
+                     "name": w.name + "+cow"})
+    return w2, np.asarray(src, dtype=np.int32), np.asarray(dst, dtype=np.int32)
+
+
 def relabel_blocks(w: Workload, perm: np.ndarray) -> Workload:
     """Same logical content with physical block b renamed perm[b] (tables and slots)."""
     perm = np.asarray(perm, dtype=np.int64)
