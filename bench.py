@@ -32,7 +32,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, SENTINEL_BF16, generate  # noqa: E402
+from workloads import CONFIGS, SENTINEL_BF16, copy_on_write_append, generate  # noqa: E402
 
 METRIC = ("paged-attn decode achieved HBM GB/s (% of B200 peak); "
           "decode steps/s at batch 64")
@@ -166,7 +166,7 @@ def prefill_bytes(w):
 
 # --------------------------------------------------------------------------- GPU arm
 class GpuRunner:
-    def __init__(self, w, torch, pa, partition_size=0, separate_store=False):
+    def __init__(self, w, torch, pa, partition_size=0, separate_store=False, cow=None):
         self.w, self.torch, self.pa = w, torch, pa
         dev = torch.device("cuda")
         shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
@@ -210,14 +210,20 @@ class GpuRunner:
         # a decode step that stores new tokens runs as one pa_store_decode call (the
         # tensor-core kernel stores the rows itself; other shapes add a store launch)
         self.fused = w.kind == "decode" and self.new_k is not None and not separate_store
+        # copy-on-write pairs copied before each step (blocks the step appends into)
+        self.cow = None if cow is None else (i32(cow[0]), i32(cow[1]))
         if self.fused and not tc:
             self.decode_launches += 1
         self.max_q = int(np.max(np.diff(w.cu_seqlens_q))) if w.num_seqs else 0
         torch.cuda.synchronize()
 
     def store(self, k=None, v=None, slots=None):
+        if self.cow is not None:
+            self.pa.pa_copy_blocks(self.k_cache, self.v_cache, *self.cow)
+            if self.fused:
+                return 1
         if self.fused or (self.new_k is None and k is None):
-            return 0
+            return 1 if self.cow is not None else 0
         self.pa.pa_store_kvcache(self.new_k if k is None else k, self.new_v if v is None else v,
                                  self.k_cache, self.v_cache, self.new_slots if slots is None else slots)
         return 1
@@ -520,9 +526,17 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
     """Device-timed numbers of the other configurations (same method, fewer steps)."""
     res = {}
     flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    for name in ("long_ctx_decode", "prefix_share_decode", "chunked_prefill"):
-        w = generate(CONFIGS[name])
-        r = GpuRunner(w, torch, pa)
+    for name in ("long_ctx_decode", "prefix_share_decode", "prefix_share_cow_append",
+                 "chunked_prefill"):
+        cow = None
+        if name == "prefix_share_cow_append":
+            # the prefix-sharing batch appending each sequence's token: the shared blocks
+            # the sequences append into are copied first, then one pa_store_decode
+            w, src, dst = copy_on_write_append(generate(CONFIGS["prefix_share_decode"]))
+            cow = (src, dst)
+        else:
+            w = generate(CONFIGS[name])
+        r = GpuRunner(w, torch, pa, cow=cow)
         n = steps if w.kind == "decode" else 50
         total_ms, attn_ms, lps = time_steps(r, torch, n, warmup, flush)
         a_ms = sum(attn_ms) / len(attn_ms)
@@ -532,7 +546,19 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
             d.update({"kernel": "pa_store_decode" if r.fused else "pa_decode", "logical_bytes": lb, "logical_GBps": round(lb / a_ms / 1e6, 1),
                       "frac_of_hbm_peak_logical": round(lb / a_ms / 1e6 / hbm_peak, 3),
                       "partition_size": r.P})
-            if name == "prefix_share_decode":
+            if cow is not None:
+                # many sequences copy the same few shared prefix blocks: the bytes the
+                # copy must move through DRAM are the distinct sources read once and
+                # every destination written (K and V)
+                blk = w.block_size * w.num_kv_heads * w.head_dim * 2
+                moved = 4 * len(cow[0]) * blk
+                dram = 2 * (len(np.unique(cow[0])) + len(cow[1])) * blk
+                c_ms = total_ms / n - a_ms
+                d.update({"copy_pairs": len(cow[0]), "copy_distinct_sources": int(len(np.unique(cow[0]))),
+                          "copy_us": round(c_ms * 1e3, 2), "copy_moved_bytes": moved,
+                          "copy_dram_bytes": dram, "copy_dram_GBps": round(dram / c_ms / 1e6, 1),
+                          "copy_frac_of_hbm_peak": round(dram / c_ms / 1e6 / hbm_peak, 3)})
+            if name.startswith("prefix_share"):
                 ub = w.kv_bytes_unique() + 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
                 d.update({"unique_bytes": ub, "unique_GBps": round(ub / a_ms / 1e6, 1),
                           "frac_of_hbm_peak_unique": round(ub / a_ms / 1e6 / hbm_peak, 3)})

@@ -92,6 +92,26 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
                            int32_t num_tokens, void* stream);
 
 /*
+ * pa_copy_blocks — copy-on-write of shared blocks. Blocks are shared between
+ * sequences by reference count (nano vllm page, section 3.2.1); the page does not
+ * say what happens when a sequence writes into a shared block, and the reading
+ * taken here is that the writer first gets a private copy, so the other sharers
+ * keep reading the unchanged block. For every i, block dst_blocks[i] of both pools
+ * becomes a copy of block src_blocks[i] (all block_size x Hkv x D values of K and
+ * of V).
+ *
+ *   src_blocks, dst_blocks  int32 [num_pairs], device. Destinations must be
+ *                  distinct and must not also be sources in the same call (the
+ *                  pairs are copied in no particular order). A pair with an id
+ *                  outside the pool is skipped and reported as PA_ERR_BAD_INDEX
+ *                  (debug checks / pa_check_device_errors); src == dst is a no-op.
+ * Moves 4 x block_size x Hkv x D x 2 bytes per pair (read and write, K and V).
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, pa_cache_desc cache,
+                         const int32_t* src_blocks, const int32_t* dst_blocks, int32_t num_pairs,
+                         void* stream);
+
+/*
  * Decode split size. The context of every sequence is cut into partitions of
  * partition_size positions (a multiple of 64); each (sequence, kv head,
  * partition) is processed independently and the partials are merged at the end

@@ -19,7 +19,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
                 4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT"}
 
 # every extern "C" function include/pa.h declares
-EXPORTED = ("pa_store_kvcache", "pa_decode_default_partition", "pa_decode_workspace_size",
+EXPORTED = ("pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
             "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
             "pa_check_device_errors", "pa_status_string", "pa_version")
 
@@ -54,6 +54,8 @@ def load_library(path: str | None = None):
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     lib.pa_store_kvcache.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp]
     lib.pa_store_kvcache.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [vp, vp, pa_cache_desc, vp, vp, i32, vp]
+    lib.pa_copy_blocks.restype = ctypes.c_int
     lib.pa_decode_default_partition.argtypes = [i32, i32, i32]
     lib.pa_decode_default_partition.restype = i32
     lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
@@ -179,6 +181,22 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                        _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
                        _stream(stream))
     _raise("pa_decode", st)
+
+
+def pa_copy_blocks(k_cache, v_cache, src_blocks, dst_blocks, stream=None) -> None:
+    """Copy-on-write: block dst_blocks[i] of both pools becomes a copy of block
+    src_blocks[i] (destinations distinct, and not also sources)."""
+    torch = _torch()
+    lib = load_library()
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(src_blocks, "src_blocks", torch.int32, 1)
+    _check(dst_blocks, "dst_blocks", torch.int32, 1)
+    if src_blocks.shape != dst_blocks.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("src/dst lengths or the two pools' shapes disagree")
+    st = lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(src_blocks),
+                            _ptr(dst_blocks), int(src_blocks.shape[0]), _stream(stream))
+    _raise("pa_copy_blocks", st)
 
 
 def pa_store_decode(new_k, new_v, slot_mapping, out, q, k_cache, v_cache, block_tables,

@@ -268,6 +268,20 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
                 stream);
 }
 
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, pa_cache_desc cache,
+                         const int32_t* src_blocks, const int32_t* dst_blocks, int32_t num_pairs,
+                         void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !src_blocks || !dst_blocks) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  return finish(launch_copy_blocks(k_cache, v_cache, cache, src_blocks, dst_blocks, num_pairs,
+                                   static_cast<cudaStream_t>(stream)),
+                stream);
+}
+
 int32_t pa_decode_default_partition(int32_t num_seqs, int32_t num_kv_heads,
                                     int32_t max_context_len) {
   // Work items are (partition, sequence, kv head) taken dynamically by one

@@ -30,6 +30,9 @@ bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uin
                           uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
                           bool swizzle128);
 
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const pa_cache_desc& c,
+                               const int32_t* src_blocks, const int32_t* dst_blocks,
+                               int32_t num_pairs, cudaStream_t stream);
 cudaError_t launch_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
                                  const pa_cache_desc& c, const int32_t* slot_mapping,
                                  int32_t num_tokens, cudaStream_t stream);

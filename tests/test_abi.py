@@ -151,3 +151,12 @@ def test_binding_store_decode_shapes():
         pa.pa_store_decode(k, k, torch.zeros(4, dtype=torch.int32), k, k, k, k,
                            torch.zeros(4, 4, dtype=torch.int32), torch.zeros(4, dtype=torch.int32),
                            0.1, 32)
+
+
+def test_copy_blocks_argument_checks(lib):
+    d = desc()
+    assert lib.pa_copy_blocks(FAKE, FAKE, d, FAKE, FAKE, -1, NULL) == 1
+    assert lib.pa_copy_blocks(NULL, FAKE, d, FAKE, FAKE, 2, NULL) == 1
+    assert lib.pa_copy_blocks(FAKE, FAKE, d, NULL, FAKE, 2, NULL) == 1
+    assert lib.pa_copy_blocks(FAKE, FAKE, desc(bs=12), FAKE, FAKE, 2, NULL) == 1
+    assert lib.pa_copy_blocks(NULL, NULL, d, NULL, NULL, 0, NULL) == 0   # no-op
