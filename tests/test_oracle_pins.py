@@ -328,3 +328,27 @@ def test_copy_on_write_append_equals_brute_force_and_keeps_sharers_intact():
         last = int(w.context_lens[s]) - 1
         shared_slots.append(int(w.block_tables[s, last // bs]) * bs + last % bs)
     assert len(set(np.array(shared_slots) // bs)) < len(shared_slots)
+
+
+# ---------------------------------------------------------------- chained block hashes
+def test_block_hashes_against_golden_and_the_recursive_rule():
+    import os
+    from workloads import compute_hash
+    golden = os.path.join(os.path.dirname(__file__), "golden", "rolling_hash.txt")
+    for line in open(golden):
+        if line.startswith("#") or not line.strip():
+            continue
+        pre, toks, want = [x.strip() for x in line.split(";")]
+        toks = [int(t) for t in toks.split()] if toks else []
+        if int(pre) == 0 and toks:
+            # a seed of 0 is the first block: the closed form over the whole block
+            assert int(oracle.block_hashes(toks, len(toks))[0]) == int(want)
+    rng = np.random.default_rng(71)
+    for bs in (1, 3, 16):
+        toks = rng.integers(0, 1 << 31, size=5 * bs + (bs - 1)).tolist()   # 5 full blocks + a tail
+        got = oracle.block_hashes(toks, bs)
+        assert len(got) == 5
+        h = 0
+        for b in range(5):
+            h = compute_hash(toks[b * bs:(b + 1) * bs], h)
+            assert int(got[b]) == h

@@ -167,3 +167,36 @@ def test_relabel_blocks_moves_slots_with_tables():
             a = int(w.block_tables[s, p // bs]) * bs + p % bs
             b = int(r.block_tables[s, p // bs]) * bs + p % bs
             assert b == perm[a // bs] * bs + a % bs
+
+
+def test_block_manager_append_fresh_private_and_shared():
+    bm = BlockManager(num_blocks=8, block_size=2, free_order=[3, 1, 4, 0, 5, 2, 6, 7])
+    a = bm.allocate([1, 2, 3])              # blocks 3 (full, hashed), 1 (partial)
+    slot, cp = bm.append(a, 3, 9)            # into the private partial block 1
+    assert (slot, cp) == (1 * 2 + 1, None) and bm.blocks[1].token_ids == [3, 9]
+    slot, cp = bm.append(a, 4, 5)            # starts a block: fresh block 4
+    assert (slot, cp) == (4 * 2, None) and a == [3, 1, 4]
+    b = bm.allocate([1, 2, 7])               # shares block 3 with a
+    assert b[0] == 3 and bm.blocks[3].ref_count == 2
+    # a second request whose partial tail reuses a cached full block, then appends to it
+    c = bm.allocate([1])                     # partial tail [1] is a prefix of block 3's tokens
+    assert c == [3] and bm.blocks[3].ref_count == 3
+    slot, cp = bm.append(c, 1, 8)            # shared: copy-on-write into a fresh block
+    assert cp == (3, c[0]) and c[0] != 3 and slot == c[0] * 2 + 1
+    assert bm.blocks[3].ref_count == 2 and bm.blocks[c[0]].token_ids == [1, 8]
+    assert bm.blocks[3].token_ids == [1, 2]  # the shared block is untouched
+
+
+def test_block_manager_append_into_private_hashed_block_forgets_its_hash():
+    bm = BlockManager(num_blocks=4, block_size=2)
+    a = bm.allocate([1, 2])                  # block 0, hashed
+    bm.free_table(a)                         # freed: hash forgotten, back on the free list
+    c = bm.allocate([1, 2])                  # block 1 (the free list continues), hashed
+    h = bm.blocks[c[0]].hash
+    d = bm.allocate([1])                     # partial tail reuses block c[0]
+    bm.free_table(c)                         # c finishes: d holds the block alone
+    assert bm.blocks[d[0]].ref_count == 1 and bm.blocks[d[0]].hash == h
+    slot, cp = bm.append(d, 1, 5)            # private but hashed: forget, write in place
+    assert cp is None and slot == d[0] * 2 + 1
+    assert bm.blocks[d[0]].hash == -1 and h not in bm.hash_to_block_id
+    assert bm.blocks[d[0]].token_ids == [1, 5]

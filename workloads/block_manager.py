@@ -152,6 +152,51 @@ class BlockManager:
                 self._forget(blk)
                 self.free.append(blk.block_id)
 
+    def append(self, table: list, pos: int, token_id: int):
+        """Decode append: the slot of position `pos` (the sequence's current length)
+        of a sequence whose blocks are `table` (updated in place), and the
+        (src, dst) block copy the step needs first, or None.
+
+        Readings (the pages share blocks by reference count and never write into a
+        shared one): a position that starts a block takes a fresh block; a block
+        other sequences also hold (ref_count > 1) is replaced by a private copy
+        (copy-on-write); a private block that is still registered under a hash is
+        dropped from the hash map before it is written (a later request must not
+        find it by a hash its contents no longer match). Blocks filled by appends
+        are not hashed.
+        """
+        bs = self.block_size
+        bi, off = divmod(int(pos), bs)
+        if bi == len(table):
+            if off:
+                raise ValueError("pos skips a block")
+            blk = self._take_free()
+            blk.ref_count = 1
+            blk.hash = -1
+            blk.token_ids = [int(token_id)]
+            table.append(blk.block_id)
+            return blk.block_id * bs, None
+        if bi > len(table) or bi < 0:
+            raise ValueError("pos outside the table")
+        blk = self.blocks[int(table[bi])]
+        copy = None
+        if blk.ref_count > 1:
+            new = self._take_free()
+            new.ref_count = 1
+            new.hash = -1
+            new.token_ids = list(blk.token_ids[:off])
+            blk.ref_count -= 1
+            copy = (blk.block_id, new.block_id)
+            table[bi] = new.block_id
+            blk = new
+        elif blk.hash != -1:
+            keep = list(blk.token_ids[:off])
+            self._forget(blk)
+            blk.token_ids = keep
+        del blk.token_ids[off:]
+        blk.token_ids.append(int(token_id))
+        return blk.block_id * bs + off, copy
+
     # -- introspection ----------------------------------------------------
     def num_used(self) -> int:
         return sum(1 for b in self.blocks if b.ref_count > 0)
