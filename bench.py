@@ -504,6 +504,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.headline_only:
         line["other_workloads"] = measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src)
+        line["block_manager"] = measure_block_manager(torch, pa)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ct, cb, n, cores, blas = cpu_oracle_time(w)
         line["cpu_baseline"] = {"value": round(cb / ct / 1e9, 4), "unit": "GB/s", "cores": cores,
@@ -576,6 +577,56 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
         del r
         torch.cuda.empty_cache()
     return res
+
+
+def measure_block_manager(torch, pa, reps=50):
+    """Prefix-sharing batch (512 requests, lognormal lengths, a shared 1024-token
+    prompt, block size 64): the batched GPU block hashes, and the host block manager
+    allocating every request's table (hashes given, and hashed on the host)."""
+    cfg = CONFIGS["prefix_share_decode"]
+    w = generate(cfg)
+    rng = np.random.default_rng(11)
+    prefix = rng.integers(1, 1 << 20, size=1024).tolist()
+    seqs = [prefix[:n] + rng.integers(1, 1 << 20, size=max(0, int(n) - 1024)).tolist()
+            for n in w.context_lens]
+    bs = cfg.block_size
+    lens = np.array([len(x) for x in seqs], dtype=np.int64)
+    toks = np.concatenate([np.asarray(x, dtype=np.int32) for x in seqs])
+    cu_t = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).cuda()
+    cu_b_h = np.concatenate([[0], np.cumsum(lens // bs)]).astype(np.int32)
+    cu_b = torch.from_numpy(cu_b_h).cuda()
+    d_t = torch.from_numpy(toks).cuda()
+    out = torch.zeros(int(cu_b_h[-1]), dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        pa.pa_block_hashes(d_t, cu_t, cu_b, bs, out)
+    torch.cuda.synchronize()
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_ev.record()
+    for _ in range(reps):
+        pa.pa_block_hashes(d_t, cu_t, cu_b, bs, out)
+    e_ev.record()
+    torch.cuda.synchronize()
+    hash_us = s_ev.elapsed_time(e_ev) * 1e3 / reps
+    hs = out.cpu().numpy().view(np.uint32)
+    per_seq = [hs[cu_b_h[i]:cu_b_h[i + 1]] for i in range(len(seqs))]
+
+    def alloc(with_hashes):
+        bm = pa.BlockManager(int(lens.sum() // bs + len(seqs) + 64), bs)
+        t0 = time.perf_counter()
+        for x, h in zip(seqs, per_seq):
+            bm.allocate(x, block_hashes=h if with_hashes else None)
+        dt = time.perf_counter() - t0
+        used = bm.num_used()
+        bm.close()
+        return dt, used
+
+    t_given, used = alloc(True)
+    t_host, _ = alloc(False)
+    return {"requests": len(seqs), "tokens": int(lens.sum()), "block_size": bs,
+            "gpu_hash_us": round(hash_us, 2), "gpu_hash_Mtokens_per_s": round(lens.sum() / hash_us, 1),
+            "host_alloc_ms_hashes_given": round(t_given * 1e3, 2),
+            "host_alloc_ms_hashing_on_host": round(t_host * 1e3, 2),
+            "blocks_used": used, "note": "host times include the ctypes call per request"}
 
 
 def run_reference(args, cfg, world):

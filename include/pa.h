@@ -60,7 +60,8 @@ typedef enum {
   PA_ERR_UNSUPPORTED = 2,
   PA_ERR_BAD_INDEX = 3,
   PA_ERR_CUDA = 4,
-  PA_ERR_TIMEOUT = 5
+  PA_ERR_TIMEOUT = 5,
+  PA_ERR_NO_BLOCKS = 6  /* block manager: the pool has no free block left */
 } pa_status;
 
 /* Shape of the paged pool (both k_cache and v_cache have this shape). */
@@ -90,6 +91,72 @@ typedef struct {
 pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_cache,
                            pa_cache_desc cache, const int32_t* slot_mapping,
                            int32_t num_tokens, void* stream);
+
+/*
+ * Host block manager (no device memory, no CUDA calls): which physical block of the
+ * pool each block of a request lives in, and which blocks requests share (nano vllm
+ * page, section 3.2: Block = id, reference count, hash, token ids; BlockManager
+ * reuses a full block whose chained hash is registered and whose tokens match, else
+ * takes a free block and registers it; section 4.2: rolling hash h = h * 31 + token
+ * mod 2^32 seeded with the previous block's hash; mini-vllm page, section 1: the
+ * BlockAllocator hands out blocks and takes them back). Readings: a trailing partial
+ * block whose prefix chain matched reuses a cached full block it is a prefix of; free
+ * blocks are taken in the order given at creation; a freed block forgets its hash.
+ * All pointers are host pointers. A manager is not thread-safe: calls on one manager
+ * must not overlap.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* num_blocks blocks of block_size positions; free_order: int32 [num_blocks], a
+ * permutation of the pool giving the order free blocks are taken (NULL = 0, 1, ...).
+ * Returns NULL for bad sizes or a free_order that is not a permutation. */
+pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order);
+void pa_bm_destroy(pa_block_manager* bm);
+
+/* The block table of one request: token_ids int32 [num_tokens] (non-negative);
+ * table_out int32 [ceil(num_tokens / block_size)]. block_hashes: NULL (hashes are
+ * computed here) or uint32 [num_tokens / block_size], the chained hash of each full
+ * block as pa_block_hashes computes it. PA_ERR_NO_BLOCKS when the pool runs out: the
+ * request then holds no block (the blocks it had taken go back to the free list). */
+pa_status pa_bm_allocate(pa_block_manager* bm, const int32_t* token_ids, int32_t num_tokens,
+                         const uint32_t* block_hashes, int32_t* table_out);
+
+/* A finished request: one reference dropped per entry; blocks reaching zero go back to
+ * the free list. An id outside the pool or a block released more often than it is held
+ * returns PA_ERR_INVALID_ARG and changes nothing. */
+pa_status pa_bm_free(pa_block_manager* bm, const int32_t* table, int32_t num_entries);
+
+/* Decode append of token_id at position pos (the sequence's current length) of a
+ * request whose table has *num_entries entries (room for capacity). Writes the slot
+ * (block * block_size + pos % block_size) to slot_out. A position that starts a block
+ * appends a fresh block to the table. A block other requests also hold is replaced by
+ * a private copy: the table entry changes and *copy_src -> *copy_dst is the copy the
+ * step must make first (pa_copy_blocks); otherwise both are -1. A private block still
+ * registered under a hash leaves the hash map before it is written. */
+pa_status pa_bm_append(pa_block_manager* bm, int32_t* table, int32_t* num_entries, int32_t capacity,
+                       int32_t pos, int32_t token_id, int32_t* slot_out, int32_t* copy_src,
+                       int32_t* copy_dst);
+
+/* Blocks with a reference count above zero (-1 for a NULL manager). */
+int32_t pa_bm_num_used(const pa_block_manager* bm);
+/* Reference count of every block: out int32 [num_blocks]. */
+pa_status pa_bm_ref_counts(const pa_block_manager* bm, int32_t* out);
+
+/*
+ * pa_block_hashes — the chained hash of every full block of a batch of token
+ * sequences on the GPU (the hash of nano vllm page, section 4.2, as above; the first
+ * block of a sequence is seeded with 0), for pa_bm_allocate. Device pointers:
+ *   token_ids   int32 [cu_tokens[num_seqs]], the sequences back to back;
+ *   cu_tokens   int32 [num_seqs + 1], token offsets;
+ *   cu_blocks   int32 [num_seqs + 1], offsets of each sequence's full blocks in
+ *               hashes_out (cu_blocks[s+1] - cu_blocks[s] = length_s / block_size);
+ *   hashes_out  uint32 [cu_blocks[num_seqs]].
+ * One warp per sequence: each lane hashes whole blocks on its own, then the lanes
+ * chain them with a scan (the chained hash of a prefix is a polynomial in 31).
+ */
+pa_status pa_block_hashes(const int32_t* token_ids, const int32_t* cu_tokens,
+                          const int32_t* cu_blocks, int32_t num_seqs, int32_t block_size,
+                          uint32_t* hashes_out, void* stream);
 
 /*
  * pa_copy_blocks — copy-on-write of shared blocks. Blocks are shared between

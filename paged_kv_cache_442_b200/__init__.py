@@ -16,10 +16,12 @@ LIB_PATH = os.path.join(PKG_DIR, "libpa.so")
 
 PA_OK = 0
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_BAD_INDEX",
-                4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT"}
+                4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT", 6: "PA_ERR_NO_BLOCKS"}
 
 # every extern "C" function include/pa.h declares
-EXPORTED = ("pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
+EXPORTED = ("pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_free", "pa_bm_append",
+            "pa_bm_num_used", "pa_bm_ref_counts", "pa_block_hashes",
+            "pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
             "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
             "pa_check_device_errors", "pa_status_string", "pa_version")
 
@@ -54,6 +56,23 @@ def load_library(path: str | None = None):
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     lib.pa_store_kvcache.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp]
     lib.pa_store_kvcache.restype = ctypes.c_int
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.pa_bm_create.argtypes = [i32, i32, vp]
+    lib.pa_bm_create.restype = vp
+    lib.pa_bm_destroy.argtypes = [vp]
+    lib.pa_bm_destroy.restype = None
+    lib.pa_bm_allocate.argtypes = [vp, vp, i32, vp, vp]
+    lib.pa_bm_allocate.restype = ctypes.c_int
+    lib.pa_bm_free.argtypes = [vp, vp, i32]
+    lib.pa_bm_free.restype = ctypes.c_int
+    lib.pa_bm_append.argtypes = [vp, vp, i32p, i32, i32, i32, i32p, i32p, i32p]
+    lib.pa_bm_append.restype = ctypes.c_int
+    lib.pa_bm_num_used.argtypes = [vp]
+    lib.pa_bm_num_used.restype = i32
+    lib.pa_bm_ref_counts.argtypes = [vp, vp]
+    lib.pa_bm_ref_counts.restype = ctypes.c_int
+    lib.pa_block_hashes.argtypes = [vp, vp, vp, i32, i32, vp, vp]
+    lib.pa_block_hashes.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, pa_cache_desc, vp, vp, i32, vp]
     lib.pa_copy_blocks.restype = ctypes.c_int
     lib.pa_decode_default_partition.argtypes = [i32, i32, i32]
@@ -181,6 +200,91 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                        _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
                        _stream(stream))
     _raise("pa_decode", st)
+
+
+class BlockManager:
+    """The library's host block manager (include/pa.h, pa_bm_*): block tables with
+    hash-chained prefix sharing, reference counts, and decode append with
+    copy-on-write. Host memory only; not thread-safe."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        import numpy as np
+        self._np = np
+        self.lib = load_library()
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+        self.h = self.lib.pa_bm_create(self.num_blocks, self.block_size,
+                                       order.ctypes.data if order is not None else None)
+        if not self.h:
+            raise ValueError("bad sizes or free_order is not a permutation of the pool")
+        self._order = order
+
+    def close(self):
+        if self.h:
+            self.lib.pa_bm_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def allocate(self, token_ids, block_hashes=None) -> list:
+        np = self._np
+        toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+        table = np.zeros(-(-len(toks) // self.block_size), dtype=np.int32)
+        hs = None if block_hashes is None else np.ascontiguousarray(block_hashes, dtype=np.uint32)
+        st = self.lib.pa_bm_allocate(self.h, toks.ctypes.data, len(toks),
+                                     hs.ctypes.data if hs is not None else None, table.ctypes.data)
+        _raise("pa_bm_allocate", st)
+        return table.tolist()
+
+    def free(self, table) -> None:
+        t = self._np.ascontiguousarray(table, dtype=self._np.int32)
+        _raise("pa_bm_free", self.lib.pa_bm_free(self.h, t.ctypes.data, len(t)))
+
+    def append(self, table: list, pos: int, token_id: int):
+        """Slot of position pos; `table` (a list) is updated in place. Returns
+        (slot, (src, dst) copy or None)."""
+        np = self._np
+        buf = np.zeros(len(table) + 1, dtype=np.int32)
+        buf[:len(table)] = table
+        n = ctypes.c_int32(len(table))
+        slot, src, dst = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+        st = self.lib.pa_bm_append(self.h, buf.ctypes.data, ctypes.byref(n), len(buf), int(pos),
+                                   int(token_id), ctypes.byref(slot), ctypes.byref(src),
+                                   ctypes.byref(dst))
+        _raise("pa_bm_append", st)
+        table[:] = buf[:n.value].tolist()
+        return slot.value, (None if src.value < 0 else (src.value, dst.value))
+
+    def num_used(self) -> int:
+        return int(self.lib.pa_bm_num_used(self.h))
+
+    def ref_counts(self):
+        out = self._np.zeros(self.num_blocks, dtype=self._np.int32)
+        _raise("pa_bm_ref_counts", self.lib.pa_bm_ref_counts(self.h, out.ctypes.data))
+        return out
+
+
+def pa_block_hashes(token_ids, cu_tokens, cu_blocks, block_size: int, hashes_out, stream=None) -> None:
+    """Chained hash of every full block of a batch of sequences (device tensors:
+    int32 tokens back to back, int32 token and block offsets, uint32-sized output)."""
+    torch = _torch()
+    lib = load_library()
+    _check(token_ids, "token_ids", torch.int32, 1)
+    _check(cu_tokens, "cu_tokens", torch.int32, 1)
+    _check(cu_blocks, "cu_blocks", torch.int32, 1)
+    _check(hashes_out, "hashes_out", hashes_out.dtype, 1)
+    if hashes_out.element_size() != 4 or cu_tokens.shape != cu_blocks.shape:
+        raise ValueError("hashes_out must hold 32-bit values; cu_tokens and cu_blocks must match")
+    st = lib.pa_block_hashes(_ptr(token_ids), _ptr(cu_tokens), _ptr(cu_blocks),
+                             int(cu_tokens.shape[0]) - 1, int(block_size), _ptr(hashes_out),
+                             _stream(stream))
+    _raise("pa_block_hashes", st)
 
 
 def pa_copy_blocks(k_cache, v_cache, src_blocks, dst_blocks, stream=None) -> None:

@@ -1,7 +1,8 @@
 """Build libpa.so in-tree with nvcc for sm_100a (B200).
 
 Usage: python -m paged_kv_cache_442_b200.build [--force] [--ptxas-verbose]
-Each .cu under csrc/ is compiled to an object in _build/ (in parallel), then the
+Each .cu (device and host code) and .cpp (host-only code) under csrc/ is compiled to
+an object in _build/ by nvcc (in parallel), then the
 objects are linked into paged_kv_cache_442_b200/libpa.so with the CUDA runtime
 linked statically. Rebuilds only when a source or header is newer than the library.
 """
@@ -32,7 +33,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():

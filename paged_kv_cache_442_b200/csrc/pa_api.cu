@@ -228,6 +228,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_BAD_INDEX: return "PA_ERR_BAD_INDEX";
     case PA_ERR_CUDA: return "PA_ERR_CUDA";
     case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT";
+    case PA_ERR_NO_BLOCKS: return "PA_ERR_NO_BLOCKS";
   }
   return "PA_ERR_UNKNOWN";
 }
@@ -265,6 +266,17 @@ pa_status pa_store_kvcache(const void* k, const void* v, void* k_cache, void* v_
     return PA_ERR_INVALID_ARG;
   return finish(launch_store_kvcache(k, v, k_cache, v_cache, cache, slot_mapping, num_tokens,
                                      static_cast<cudaStream_t>(stream)),
+                stream);
+}
+
+pa_status pa_block_hashes(const int32_t* token_ids, const int32_t* cu_tokens,
+                          const int32_t* cu_blocks, int32_t num_seqs, int32_t block_size,
+                          uint32_t* hashes_out, void* stream) {
+  if (num_seqs < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!token_ids || !cu_tokens || !cu_blocks || !hashes_out) return PA_ERR_INVALID_ARG;
+  return finish(launch_block_hashes(token_ids, cu_tokens, cu_blocks, num_seqs, block_size,
+                                    hashes_out, static_cast<cudaStream_t>(stream)),
                 stream);
 }
 

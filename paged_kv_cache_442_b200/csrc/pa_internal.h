@@ -30,6 +30,9 @@ bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uin
                           uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
                           bool swizzle128);
 
+cudaError_t launch_block_hashes(const int32_t* token_ids, const int32_t* cu_tokens,
+                                const int32_t* cu_blocks, int32_t num_seqs, int32_t block_size,
+                                uint32_t* hashes_out, cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const pa_cache_desc& c,
                                const int32_t* src_blocks, const int32_t* dst_blocks,
                                int32_t num_pairs, cudaStream_t stream);
