@@ -421,7 +421,7 @@ def main():
 
     hbm_peak, tf_peak, tf_sustained, peak_src = peaks()
     # every rank decodes its own batch of the same shape (weak scaling)
-    w = generate(cfg) if rank == 0 else _rank_workload(cfg, rank)
+    w = rank_workload(cfg, rank)
     runner = GpuRunner(w, torch, pa, args.partition_size, args.separate_store)
     flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
@@ -434,13 +434,10 @@ def main():
     t1 = time.time()
     clocks = sampler.stop(t0, t1)
 
-    step_ms = total_ms / args.steps
-    if pg is not None:
-        t = torch.tensor([step_ms], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(total_ms / args.steps, pg, torch, "cuda")
     bytes_step = (decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)) + store_bytes(w)
-    value = world * bytes_step / (step_ms * 1e-3) / 1e9
+    job_bytes = sum_over_ranks(bytes_step, pg, torch, "cuda")
+    value = job_gbps(job_bytes, step_ms)
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
     if runner.fused:
@@ -466,7 +463,7 @@ def main():
                     "traffic": recorded_traffic(cfg.name + ".prefill", PREFILL_SRC)}
 
     e2e_ms, h2d, d2h = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
-    e2e_step_ms = e2e_ms / min(args.steps, 500)
+    e2e_step_ms = max_over_ranks(e2e_ms / min(args.steps, 500), pg, torch, "cuda")
 
     line = {
         "metric": METRIC,
@@ -493,7 +490,7 @@ def main():
         "pct_of_datasheet_8tbs": round(100 * value / world / DATASHEET_HBM_GBS, 1),
         "bytes_per_step": bytes_step,
         "roofline": roofline,
-        "e2e": {"value": round(world * bytes_step / (e2e_step_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(job_gbps(job_bytes, e2e_step_ms), 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_step_ms, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "api": ("paged_kv_cache_442_b200.pa_store_decode" if runner.fused else
@@ -518,9 +515,36 @@ def main():
         print(json.dumps(line), flush=True)
 
 
-def _rank_workload(cfg, rank):
+def rank_workload(cfg, rank):
+    """Rank r's batch: the same configuration (shape) drawn from another seed, so the
+    ranks decode independent sequences (weak scaling; rank 0's batch is the
+    configuration's own)."""
     from dataclasses import replace
     return generate(replace(cfg, index=cfg.index + 100 * rank))
+
+
+def max_over_ranks(x, dist, torch, device):
+    """The slowest rank's value (every rank gets it); x itself when not distributed."""
+    if dist is None:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, dist, torch, device):
+    """Sum over ranks (every rank gets it); x itself when not distributed."""
+    if dist is None:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_gbps(job_bytes, step_ms):
+    """Whole-job throughput: the bytes all ranks moved in a step over the slowest
+    rank's step time."""
+    return job_bytes / (step_ms * 1e-3) / 1e9
 
 
 def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=200, warmup=10):
