@@ -250,6 +250,99 @@ class GpuRunner:
         return self.store() + self.attend()
 
 
+def fp8_decode_bytes(w):
+    """Bytes an fp8 decode reads and writes: the e4m3 codes and the fp32 row scales of K
+    and V at every position of every sequence, q in and the output out."""
+    pos = int(w.context_lens.astype(np.int64).sum())
+    kv = pos * w.num_kv_heads * (w.head_dim + 4) * 2
+    qo = 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+    return kv + qo
+
+
+def fp8_store_bytes(w):
+    """Bytes the fp8 store moves: bf16 rows in, codes and scales out (K and V)."""
+    return len(w.new_slots) * w.num_kv_heads * (2 * w.head_dim + w.head_dim + 4) * 2
+
+
+class Fp8Runner:
+    """A decode step over e4m3 pools: the step's new rows quantised into the pools
+    (pa_store_kvcache_fp8), then pa_decode_fp8. The cached context is quantised by the
+    same store during setup (untimed); unwritten rows hold NaN codes and scales."""
+
+    def __init__(self, w, torch, pa):
+        self.w, self.pa = w, pa
+        dev = torch.device("cuda")
+        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        self.k8 = torch.full(shape, 0x7F, dtype=torch.uint8, device=dev)
+        self.v8 = torch.full(shape, 0x7F, dtype=torch.uint8, device=dev)
+        sshape = (w.num_kv_heads, w.num_blocks * w.block_size)
+        self.ks = torch.full(sshape, float("nan"), dtype=torch.float32, device=dev)
+        self.vs = torch.full(sshape, float("nan"), dtype=torch.float32, device=dev)
+
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        def i32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+        n = len(w.setup_slots)
+        for s0 in range(0, n, 1 << 18):
+            idx = np.arange(s0, min(n, s0 + (1 << 18)))
+            pa.pa_store_kvcache_fp8(bf(w.src_k[w.setup_src[idx]]), bf(w.src_v[w.setup_src[idx]]),
+                                    self.k8, self.v8, self.ks, self.vs, i32(w.setup_slots[idx]))
+        self.q = bf(w.q)
+        self.new_k = bf(w.new_k) if len(w.new_slots) else None
+        self.new_v = bf(w.new_v) if len(w.new_slots) else None
+        self.new_slots = i32(w.new_slots)
+        self.block_tables = i32(w.block_tables)
+        self.context_lens = i32(w.context_lens)
+        self.out = torch.empty_like(self.q)
+        self.ws, self.P = pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads,
+                                              w.head_dim, w.max_context_len)
+        torch.cuda.synchronize()
+
+    def store(self):
+        if self.new_k is None:
+            return 0
+        self.pa.pa_store_kvcache_fp8(self.new_k, self.new_v, self.k8, self.v8, self.ks, self.vs,
+                                     self.new_slots)
+        return 1
+
+    def attend(self):
+        w = self.w
+        self.pa.pa_decode_fp8(self.out, self.q, self.k8, self.v8, self.ks, self.vs,
+                              self.block_tables, self.context_lens, w.scale, w.max_context_len,
+                              self.P, self.ws)
+        return 1
+
+    def step(self):
+        return self.store() + self.attend()
+
+
+def measure_fp8_decode(torch, pa, hbm_peak, peak_src, bf16_attn_us, steps=200, warmup=10):
+    """The headline decode batch over e4m3 pools (same sequences, same step shape)."""
+    w = generate(CONFIGS["decode_b64"])
+    r = Fp8Runner(w, torch, pa)
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    total_ms, attn_ms, lps = time_steps(r, torch, steps, warmup, flush)
+    a_ms = sum(attn_ms) / len(attn_ms)
+    st_ms = total_ms / steps - a_ms
+    b = fp8_decode_bytes(w)
+    d = {"kernel": "pa_decode_fp8 (persistent tcgen05 decode, e4m3 tiles dequantised in "
+                   "shared memory)", "attn_us": round(a_ms * 1e3, 2),
+         "step_us": round(total_ms / steps * 1e3, 2), "steps": steps, "launches_per_step": lps,
+         "algorithmic_bytes": b, "GBps": round(b / a_ms / 1e6, 1),
+         "frac_of_hbm_peak": round(b / a_ms / 1e6 / hbm_peak, 3),
+         "store_us": round(st_ms * 1e3, 2),
+         "store_GBps": round(fp8_store_bytes(w) / st_ms / 1e6, 1) if st_ms > 0 else None,
+         "partition_size": r.P, "peak_source": peak_src}
+    if bf16_attn_us:
+        d["attn_time_vs_bf16_store_decode"] = round(a_ms * 1e3 / bf16_attn_us, 3)
+    del r
+    torch.cuda.empty_cache()
+    return d
+
+
 def time_steps(runner, torch, steps, warmup, flush_buf, barrier=None):
     """Per-step device time (ms) of `steps` steps, L2 flushed before each step.
 
@@ -501,6 +594,9 @@ def main():
     }
     if rank == 0 and world == 1 and not args.headline_only:
         line["other_workloads"] = measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src)
+        if cfg.name == "decode_b64":
+            line["other_workloads"]["decode_b64_fp8"] = measure_fp8_decode(
+                torch, pa, hbm_peak, peak_src, attn_avg_ms * 1e3)
         line["block_manager"] = measure_block_manager(torch, pa)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ct, cb, n, cores, blas = cpu_oracle_time(w)

@@ -299,6 +299,52 @@ pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_cache, cons
                              int32_t max_context_len, int32_t partition_size, void* stream);
 
 /*
+ * fp8 (e4m3) KV cache. The nano vllm KV-cache practice page lists quantisation
+ * support among its extensions (section 5.3 "扩展建议") and the Nano-vLLM
+ * architecture page names quantised compression as a further direction (section 7
+ * "总结与展望"); neither fixes a format, so the readings taken here are:
+ *  - values are OCP fp8 e4m3 codes (bias 7, no infinities, largest finite 448);
+ *  - every (pool row, kv head) pair of D values has its own fp32 scale, chosen when
+ *    the row is written (a decode step writes one row of a block at a time, so a
+ *    per-block scale could not be fixed before the block is full);
+ *  - a row x is quantised in fp32: amax = max |x|; amax == 0 gives codes 0 and
+ *    scale 0; else code_i = e4m3(x_i * (448 / amax)), rounded to nearest even and
+ *    saturated to +-448, and scale = amax / 448 (both divisions rounded to nearest);
+ *  - a stored value reads back as e4m3(code) * scale.
+ * Pools: codes uint8 [num_blocks, block_size, Hkv, D] (the bf16 pool's row
+ * layout with one byte per value); scales fp32 [Hkv, num_blocks * block_size]
+ * (kv head major: the scales of one kv head's consecutive pool rows are
+ * contiguous). Halves the bytes a decode step reads.
+ */
+
+/*
+ * pa_store_kvcache_fp8 — pa_store_kvcache into e4m3 pools: row slot_mapping[t] of
+ * k_codes / v_codes receives the quantised k[t] / v[t] and k_scales / v_scales
+ * [g][slot_mapping[t]] the scale of kv head g's row. k, v: [num_tokens, Hkv, D]
+ * bf16. Skipped and bad slots as in pa_store_kvcache. head_dim 64 or 128.
+ */
+pa_status pa_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void* v_codes,
+                               float* k_scales, float* v_scales, pa_cache_desc cache,
+                               const int32_t* slot_mapping, int32_t num_tokens, void* stream);
+
+/*
+ * pa_decode_fp8 — pa_decode over e4m3 pools: the attention of the values the
+ * pools hold (code * scale). Each K/V tile is loaded as codes and scales,
+ * dequantised to bf16 (code * scale rounded once to nearest even) in shared memory,
+ * and then takes pa_decode's tensor-core path unchanged. Arguments as pa_decode,
+ * with the pools replaced by codes and scales (16-byte aligned).
+ * Supported: head_dim 128, Hq / Hkv in {1, 2, 4, 8}, partition_size (given or
+ * automatic) a multiple of 128 up to 2048; anything else returns
+ * PA_ERR_UNSUPPORTED (there is no CUDA-core fp8 path).
+ */
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_codes, const void* v_codes,
+                        const float* k_scales, const float* v_scales, pa_cache_desc cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                        float scale, int32_t max_context_len, int32_t partition_size,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pa_prefill — causal attention of a chunk of new tokens appended to each
  * sequence's cached prefix (nano vllm page, section 3.1: num_cached_tokens of a
  * Sequence are reused; mini-vllm page, section 1: blocks are allocated for the

@@ -8,10 +8,12 @@ The pages list quantisation of the KV cache only as an extension; the readings h
   * every (position, kv head) row of D values has its own fp32 scale: a decode step
     writes one row at a time into a block, so a scale per row can be chosen when the
     row is written (a per-block scale could not, before the block is full);
-  * quantising a row x (bf16 values): amax = max |x|; if amax == 0 the codes and the
-    scale are 0; otherwise, in fp32 with round-to-nearest, inv = 448 / amax,
-    y_i = x_i * inv, code_i = e4m3(y_i) rounded to nearest even and saturated to
-    +-448, and scale = amax / 448. A value is read back as e4m3(code) * scale.
+  * quantising a row x (bf16 values, finite): amax = max |x|; in fp32 with
+    round-to-nearest, inv = 448 / amax; if inv is not a finite fp32 (amax == 0, or
+    amax below 448 / FLT_MAX, about 1.3e-36, where the quotient overflows) the codes
+    and the scale are 0; otherwise y_i = x_i * inv, code_i = e4m3(y_i) rounded to
+    nearest even and saturated to +-448, and scale = amax / 448. A value is read back
+    as e4m3(code) * scale.
 The quantiser's integer decisions are taken in fp32, the precision the kernels use.
 """
 from __future__ import annotations
@@ -75,9 +77,10 @@ def quantize_rows(x_bits: np.ndarray):
     scales = np.zeros(flat.shape[0], dtype=np.float32)
     for i, row in enumerate(flat):
         amax = np.float32(np.max(np.abs(row)))
-        if amax == 0:
+        with np.errstate(over="ignore", divide="ignore"):
+            inv = np.float32(E4M3_MAX) / amax
+        if not np.isfinite(inv):
             continue
-        inv = np.float32(E4M3_MAX) / amax
         y = (row * inv).astype(np.float32)
         codes[i] = [float_to_e4m3(v) for v in y.astype(np.float64)]
         scales[i] = amax / np.float32(E4M3_MAX)

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
 EXPORTED = ("pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_free", "pa_bm_append",
             "pa_bm_num_used", "pa_bm_ref_counts", "pa_block_hashes",
             "pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
-            "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill", "pa_set_debug_checks",
+            "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill",
+            "pa_store_kvcache_fp8", "pa_decode_fp8", "pa_set_debug_checks",
             "pa_check_device_errors", "pa_status_string", "pa_version")
 
 # size of the library-owned scratch of pa_decode_no_alloc (include/pa.h)
@@ -91,6 +92,11 @@ def load_library(path: str | None = None):
     lib.pa_prefill.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, vp, i32, i32, i32, i32,
                                ctypes.c_float, vp]
     lib.pa_prefill.restype = ctypes.c_int
+    lib.pa_store_kvcache_fp8.argtypes = [vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp]
+    lib.pa_store_kvcache_fp8.restype = ctypes.c_int
+    lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
+                                  ctypes.c_float, i32, i32, vp, sz, vp]
+    lib.pa_decode_fp8.restype = ctypes.c_int
     lib.pa_set_debug_checks.argtypes = [ctypes.c_int]
     lib.pa_set_debug_checks.restype = None
     lib.pa_check_device_errors.argtypes = [vp]
@@ -200,6 +206,64 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                        _ptr(workspace) if workspace is not None else ctypes.c_void_p(0), ws_bytes,
                        _stream(stream))
     _raise("pa_decode", st)
+
+
+def _check_fp8_pools(torch, k_codes, v_codes, k_scales, v_scales):
+    _check(k_codes, "k_codes", torch.uint8, 4)
+    _check(v_codes, "v_codes", torch.uint8, 4)
+    _check(k_scales, "k_scales", torch.float32, 2)
+    _check(v_scales, "v_scales", torch.float32, 2)
+    nb, bs, hkv, _ = k_codes.shape
+    if k_codes.shape != v_codes.shape or k_scales.shape != v_scales.shape:
+        raise ValueError("K and V pools must have the same shapes")
+    if tuple(k_scales.shape) != (hkv, nb * bs):
+        raise ValueError("scales must be [num_kv_heads, num_blocks * block_size] fp32")
+
+
+def pa_store_kvcache_fp8(k, v, k_codes, v_codes, k_scales, v_scales, slot_mapping,
+                         stream=None) -> None:
+    """Quantise k[t], v[t] (bf16) into the e4m3 pools at row slot_mapping[t]: codes
+    uint8 [num_blocks, bs, Hkv, D], per-row scales fp32 [Hkv, num_blocks * bs]."""
+    torch = _torch()
+    lib = load_library()
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check_fp8_pools(torch, k_codes, v_codes, k_scales, v_scales)
+    _check(slot_mapping, "slot_mapping", torch.int32, 1)
+    if k.shape != v.shape or k.shape[0] != slot_mapping.shape[0] or \
+            tuple(k.shape[1:]) != tuple(k_codes.shape[2:]):
+        raise ValueError("k must be [num_tokens, num_kv_heads, head_dim] matching the pool")
+    st = lib.pa_store_kvcache_fp8(_ptr(k), _ptr(v), _ptr(k_codes), _ptr(v_codes), _ptr(k_scales),
+                                  _ptr(v_scales), cache_desc(k_codes), _ptr(slot_mapping),
+                                  int(k.shape[0]), _stream(stream))
+    _raise("pa_store_kvcache_fp8", st)
+
+
+def pa_decode_fp8(out, q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens,
+                  scale: float, max_context_len: int, partition_size: int = 0, workspace=None,
+                  stream=None) -> None:
+    """Paged decode attention over e4m3 pools into `out` [num_seqs, Hq, D] (bf16)."""
+    torch = _torch()
+    lib = load_library()
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check_fp8_pools(torch, k_codes, v_codes, k_scales, v_scales)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    if tuple(out.shape) != (B, Hq, D) or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("out/q/block_tables/context_lens disagree on num_seqs")
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scales),
+                           _ptr(v_scales), cache_desc(k_codes), _ptr(block_tables),
+                           int(block_tables.shape[1]), _ptr(context_lens), int(B), int(Hq),
+                           float(scale), int(max_context_len), int(partition_size),
+                           _ptr(workspace) if workspace is not None else ctypes.c_void_p(0),
+                           ws_bytes, _stream(stream))
+    _raise("pa_decode_fp8", st)
 
 
 class BlockManager:

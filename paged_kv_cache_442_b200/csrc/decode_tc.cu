@@ -37,7 +37,20 @@
 //           merges them (split-K merge in the same kernel).
 // Counters in the workspace carry a per-call tag, so an earlier call's leftovers never
 // count: the workspace needs no clearing between calls.
+//
+// fp8 variant (pa_decode_fp8): the pools hold e4m3 codes with one fp32 scale per
+// (position, kv head) row. The producer loads a tile's codes into the upper half of
+// its 32 KB ring slot and the tile's scales (one box per block, each on a 128-byte
+// boundary) into the lower half; warps 11-14 (converters) dequantise it in place:
+// thread r reads its row's 128 codes and its scale into registers, the 128 converter
+// threads meet at a named barrier (the scales sit where the first rows of the lower
+// half are written), and thread r writes its row as
+// bf16 (code * scale, rounded once) into both swizzled halves -- the upper-half write
+// covers exactly its own source row. The score, softmax, value and merge stages are
+// the bf16 ones, unchanged.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <atomic>
 #include <ctime>
@@ -60,6 +73,8 @@ constexpr int QS = 2;          // scheduler queue depth: one item prepared ahead
                                // queues reserve work early and unbalance the tail)
 constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flight)
 constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
+constexpr int kThreadsF8 = 480;  // + converters 11-14 (fp8 pools)
+constexpr int kConvWarp0 = 11;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more than this
 constexpr int kRegion = TM * 128;            // 64 head dims x 128 positions (16 KB)
 constexpr int kTileBytes = 2 * kRegion;      // one K or V tile (32 KB)
@@ -84,7 +99,7 @@ constexpr int kOffDesc = align_up(kOffSchedFb + QS * 4, 16);         // [QN] ite
 constexpr int kOffEpi = align_up(kOffDesc + QN * 32, 16);            // [NO] hand-offs
 constexpr int kEpiBytes = 32 + 2 * NQ * 4;                           // descriptor, m, l
 constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
-constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS;
+constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS + NK + NV;
 constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
@@ -235,6 +250,48 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 2-D tiled tensor load global -> shared (the fp8 scales: [Hkv][slots] fp32).
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// two fp32 products in one instruction (sm_100 packed fp32), each rounded to nearest
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float s) {
+  uint64_t r;
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "mov.b64 rb, {%3, %3};\n\t"
+      "mul.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(r)
+      : "f"(a.x), "f"(a.y), "f"(s));
+  float2 o;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+  return o;
+}
+
+// 16 e4m3 codes (one uint4, code i in byte i) times a scale -> 16 bf16 values as two
+// uint4 (values 0-7, 8-15; element i in the low half of word i/2 ... as bf16 pairs).
+// e4m3 -> f16 is exact, so code * scale is rounded once (fp32 product, then to bf16).
+__device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t out[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t two =
+        static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
+    const float2 f = mul_f32x2(__half22float2(*reinterpret_cast<const __half2*>(&h)), scale);
+    out[i] = pack_bf16x2(f.x, f.y);
+  }
+  lo = make_uint4(out[0], out[1], out[2], out[3]);
+  hi = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -248,10 +305,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
+template <int G, bool F8>
+__global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-    const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmSK,
+    const __grid_constant__ CUtensorMap tmSV, const TcParams p) {
   static_assert(G >= 1 && G <= NQ, "query heads per kv head");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -279,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   uint64_t* epi_empty = epi_full + NO;         // [NO] epilogue read the hand-off
   uint64_t* sched_full = epi_empty + NO;       // [QS] scheduler -> producer
   uint64_t* sched_empty = sched_full + QS;     // [QS] producer done with a queued item
+  uint64_t* kst_full = sched_empty + QS;       // [NK] fp8: codes + scales of K landed
+  uint64_t* vst_full = kst_full + NK;          // [NV] fp8: codes + scales of V landed
   ItemDesc* sched_desc = reinterpret_cast<ItemDesc*>(smem + kOffSched);
   int* sched_fb = reinterpret_cast<int*>(smem + kOffSchedFb);
   ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + kOffDesc);
@@ -287,19 +347,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
+  volatile int* conv_stop = reinterpret_cast<volatile int*>(smem + kOffMisc + 32);  // [NK], fp8
 
   // zero the Q slots and P^T buffers: rows >= G are never written and stay zero
-  for (int i = tid; i < (QN * kQBytes + NP * kPBytes) / 16; i += kThreads)
+  for (int i = tid; i < (QN * kQBytes + NP * kPBytes) / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
+    // fp8: a ring slot is full once the four converter warps have written it
     for (int i = 0; i < NK; ++i) {
-      mbar_init(&k_full[i], 1);
+      mbar_init(&k_full[i], F8 ? 4 : 1);
       mbar_init(&k_empty[i], 1);
+      mbar_init(&kst_full[i], 1);
+      conv_stop[i] = 0;
     }
     for (int i = 0; i < NV; ++i) {
-      mbar_init(&v_full[i], 1);
+      mbar_init(&v_full[i], F8 ? 4 : 1);
       mbar_init(&v_empty[i], 1);
+      mbar_init(&vst_full[i], 1);
     }
     for (int i = 0; i < QN; ++i) {
       mbar_init(&item_full[i], 1);
@@ -348,9 +413,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
+      if (F8) {
+        prefetch_tensormap(&tmSK);
+        prefetch_tensormap(&tmSV);
+      }
     }
     const int rows = bs < TM ? bs : TM;
     const int nbox = TM / rows;
+    // fp8: each box's scales start on a 128-byte boundary of the slot
+    const int sstride = rows * 4 < 128 ? 128 : rows * 4;
     int q = 0;       // items taken from the scheduler queue
     int k = 0;       // items published to the issuer / softmax
     unsigned j = 0;  // tiles issued
@@ -366,6 +437,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (lane == 0) {
           descs[slot] = cur;
           mbar_arrive(&item_full[slot]);
+        }
+        if (F8) {
+          // the converters follow the tile sequence: mark the next K slot as the end
+          const int ks = j % NK;
+          if (j < NK || wwait(&k_empty[ks], ((j / NK) - 1) & 1)) {
+            if (lane == 0) {
+              conv_stop[ks] = 1;
+              mbar_arrive(&kst_full[ks]);
+            }
+          }
         }
         break;
       }
@@ -412,13 +493,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         }
         if (lane == 0) {
           uint8_t* kdst = smem + kOffK + ks * kTileBytes;
-          mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
-          for (int b = 0; b < nbox; ++b) {
-            const int pos = t0 + i * TM + b * rows;
-            const int bi = (pos >> p.bs_log2) - first_blk;
-            const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
-            tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
-            tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &k_full[ks], 64, g, row);
+          if (F8) {
+            // codes into the upper half of the slot, scales into its first 512 bytes
+            mbar_arrive_expect_tx(&kst_full[ks], kRegion + TM * 4);
+            for (int b = 0; b < nbox; ++b) {
+              const int pos = t0 + i * TM + b * rows;
+              const int bi = (pos >> p.bs_log2) - first_blk;
+              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+              tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &kst_full[ks], 0, g, row);
+              tma_load_2d(kdst + b * sstride, &tmSK, &kst_full[ks], row, g);
+            }
+          } else {
+            mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
+            for (int b = 0; b < nbox; ++b) {
+              const int pos = t0 + i * TM + b * rows;
+              const int bi = (pos >> p.bs_log2) - first_blk;
+              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+              tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
+              tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &k_full[ks], 64, g, row);
+            }
           }
         }
         __syncwarp();
@@ -430,13 +523,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         }
         if (lane == 0) {
           uint8_t* vdst = smem + kOffV + vs * kTileBytes;
-          mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
-          for (int b = 0; b < nbox; ++b) {
-            const int pos = t0 + i * TM + b * rows;
-            const int bi = (pos >> p.bs_log2) - first_blk;
-            const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
-            tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
-            tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &v_full[vs], 64, g, row);
+          if (F8) {
+            mbar_arrive_expect_tx(&vst_full[vs], kRegion + TM * 4);
+            for (int b = 0; b < nbox; ++b) {
+              const int pos = t0 + i * TM + b * rows;
+              const int bi = (pos >> p.bs_log2) - first_blk;
+              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+              tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &vst_full[vs], 0, g, row);
+              tma_load_2d(vdst + b * sstride, &tmSV, &vst_full[vs], row, g);
+            }
+          } else {
+            mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
+            for (int b = 0; b < nbox; ++b) {
+              const int pos = t0 + i * TM + b * rows;
+              const int bi = (pos >> p.bs_log2) - first_blk;
+              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+              tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
+              tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &v_full[vs], 64, g, row);
+            }
           }
         }
         __syncwarp();
@@ -822,6 +926,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       if (bar_or(2, 128, failed)) break;  // also orders last_flag's reuse
       ++k;
     }
+  } else if (F8) {
+    // ======================================================== converter warps 11-14
+    // Follow the tile sequence of the producer; thread r dequantises row r of each K
+    // and V tile in place. Every thread waits on its own; the barrier vote that follows
+    // both lets them leave together and keeps every write behind every read of the
+    // slot's scales (which lie where the first rows of the lower half are written).
+    const int r = tid - kConvWarp0 * 32;
+    const int sw = r & 7;
+    // where the producer put row r's scale: box r / rows, 128-byte aligned boxes
+    const int rows = bs < TM ? bs : TM;
+    const int soff = (r / rows) * (rows * 4 < 128 ? 128 : rows * 4) + (r % rows) * 4;
+    // stop_slot: the K ring slot whose end-of-tiles mark to honour, or -1 (V tiles)
+    auto convert = [&](uint8_t* slot, uint64_t* staged, unsigned parity, uint64_t* full,
+                       int stop_slot) -> bool {
+      bool ok = wait_or_abort(staged, parity, p.err, abort_flag);
+      const bool stop = ok && stop_slot >= 0 && conv_stop[stop_slot] != 0;
+      uint4 raw[8];
+      float sc = 0.f;
+      if (ok && !stop) {
+        // chunk c ^ (r % 8) of the row in step c: the 8 threads of a quarter warp read
+        // 8 different 16-byte bank groups (rows are 128 bytes apart)
+        const uint4* src = reinterpret_cast<const uint4*>(slot + kRegion + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) raw[c] = src[c ^ sw];
+        sc = *reinterpret_cast<const float*>(slot + soff);
+      }
+      if (bar_or(3, 128, !ok || stop)) return false;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 lo, hi;
+        dequant16(raw[c], sc, lo, hi);
+        // dims 16k..16k+15 (k = c ^ (r % 8)) = 16-byte bf16 chunks 2k and 2k+1 of the
+        // row; chunk q lies in half q / 8 at position (q % 8) ^ (r % 8) (128-byte
+        // swizzle). For each (c, h) the quarter warp's 8 positions are distinct.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int q = 2 * (c ^ sw) + h;
+          uint4* dst = reinterpret_cast<uint4*>(slot + (q >> 3) * kRegion + r * 128 +
+                                                (((q & 7) ^ sw) << 4));
+          *dst = h ? hi : lo;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full);
+      return true;
+    };
+    for (unsigned j = 0;; ++j) {
+      const int ks = j % NK;
+      if (!convert(smem + kOffK + ks * kTileBytes, &kst_full[ks], (j / NK) & 1, &k_full[ks], ks))
+        break;
+      const int vs = j % NV;
+      if (!convert(smem + kOffV + vs * kTileBytes, &vst_full[vs], (j / NV) & 1, &v_full[vs], -1))
+        break;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -846,23 +1005,42 @@ unsigned long long next_tag() {
   return v;
 }
 
-template <int G>
+template <int G, bool F8>
 cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t stream) {
   const int bs = a.cache.block_size;
   const int rows = bs < TM ? bs : TM;
   const uint64_t slots = static_cast<uint64_t>(a.cache.num_blocks) * bs;
-  CUtensorMap tmQ, tmK, tmV;
-  if (!encode_tensor_map_3d(&tmQ, a.q, HD, a.num_q_heads, a.num_seqs, 64, G, 1, true) ||
-      !encode_tensor_map_3d(&tmK, a.k_cache, HD, a.cache.num_kv_heads, slots, 64, 1, rows, true) ||
-      !encode_tensor_map_3d(&tmV, a.v_cache, HD, a.cache.num_kv_heads, slots, 64, 1, rows, true))
+  const uint64_t hkv = static_cast<uint64_t>(a.cache.num_kv_heads);
+  CUtensorMap tmQ, tmK, tmV, tmSK, tmSV;
+  if (!encode_tensor_map_3d(&tmQ, a.q, HD, a.num_q_heads, a.num_seqs, 64, G, 1, true))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      ensure_max_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<G>), kSmemBytes);
+  if (F8) {
+    // codes [slots][Hkv][D] bytes, one 128-byte row per box row, no swizzle;
+    // scales [Hkv][slots] fp32, a run of `rows` positions of one kv head per box
+    const uint64_t cd[3] = {HD, hkv, slots};
+    const uint32_t cb[3] = {HD, 1, static_cast<uint32_t>(rows)};
+    const uint64_t sd[2] = {slots, hkv};
+    const uint32_t sb[2] = {static_cast<uint32_t>(rows), 1};
+    if (!encode_tensor_map(&tmK, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, false) ||
+        !encode_tensor_map(&tmV, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, false) ||
+        !encode_tensor_map(&tmSK, a.k_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, sd, sb, false) ||
+        !encode_tensor_map(&tmSV, a.v_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, sd, sb, false))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!encode_tensor_map_3d(&tmK, a.k_cache, HD, hkv, slots, 64, 1, rows, true) ||
+        !encode_tensor_map_3d(&tmV, a.v_cache, HD, hkv, slots, 64, 1, rows, true))
+      return cudaErrorInvalidValue;
+    tmSK = tmQ;  // unused by the bf16 kernel
+    tmSV = tmQ;
+  }
+  cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<G, F8>),
+                                          kSmemBytes);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  decode_tc_kernel<G><<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  decode_tc_kernel<G, F8><<<grid, F8 ? kThreadsF8 : kThreads, kSmemBytes, stream>>>(
+      tmQ, tmK, tmV, tmSK, tmSV, p);
   return cudaGetLastError();
 }
 
@@ -870,8 +1048,14 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
 
 bool decode_tc_supported(const DecodeLaunch& a) {
   const int G = a.num_q_heads / a.cache.num_kv_heads;
-  return a.cache.head_dim == HD && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16) &&
-         a.partition_size % TM == 0 && a.partition_size <= 2048;
+  // fp8 pools add four converter warps (480 threads): up to 8 query heads per kv head
+  const bool g_ok = a.fp8 ? (G == 1 || G == 2 || G == 4 || G == 8)
+                          : (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
+  // fp8 scale boxes start at slot index (block id * block size): a multiple of four
+  // fp32 (16 bytes) only when the block size is
+  const bool bs_ok = !a.fp8 || a.cache.block_size % 4 == 0;
+  return a.cache.head_dim == HD && g_ok && bs_ok && a.partition_size % TM == 0 &&
+         a.partition_size <= 2048;
 }
 
 cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters,
@@ -900,12 +1084,21 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
   p.slot_mapping = a.slot_mapping;
   p.k_rows = static_cast<uint4*>(const_cast<void*>(a.k_cache));
   p.v_rows = static_cast<uint4*>(const_cast<void*>(a.v_cache));
+  if (a.fp8) {
+    switch (a.num_q_heads / a.cache.num_kv_heads) {
+      case 1: return launch_tc_t<1, true>(a, p, stream);
+      case 2: return launch_tc_t<2, true>(a, p, stream);
+      case 4: return launch_tc_t<4, true>(a, p, stream);
+      case 8: return launch_tc_t<8, true>(a, p, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (a.num_q_heads / a.cache.num_kv_heads) {
-    case 1: return launch_tc_t<1>(a, p, stream);
-    case 2: return launch_tc_t<2>(a, p, stream);
-    case 4: return launch_tc_t<4>(a, p, stream);
-    case 8: return launch_tc_t<8>(a, p, stream);
-    case 16: return launch_tc_t<16>(a, p, stream);
+    case 1: return launch_tc_t<1, false>(a, p, stream);
+    case 2: return launch_tc_t<2, false>(a, p, stream);
+    case 4: return launch_tc_t<4, false>(a, p, stream);
+    case 8: return launch_tc_t<8, false>(a, p, stream);
+    case 16: return launch_tc_t<16, false>(a, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -99,9 +99,10 @@ cudaError_t ensure_max_dynamic_smem(const void* func, int bytes) {
   return e;
 }
 
-bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1,
-                          uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
-                          bool swizzle128) {
+bool encode_tensor_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                       int elem_bytes, int rank, const uint64_t* dims, const uint32_t* box,
+                       bool swizzle128) {
+  if (rank < 1 || rank > 5) return false;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_encode) {
@@ -114,15 +115,29 @@ bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uin
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
   }
-  const cuuint64_t dims[3] = {dim0, dim1, dim2};
-  const cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};  // bytes, dims 1 and 2
-  const cuuint32_t box[3] = {box0, box1, box2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t gdims[5], strides[4];
+  cuuint32_t gbox[5], estr[5];
+  uint64_t stride = static_cast<uint64_t>(elem_bytes);
+  for (int i = 0; i < rank; ++i) {
+    gdims[i] = dims[i];
+    gbox[i] = box[i];
+    estr[i] = 1;
+    if (i > 0) strides[i - 1] = stride;  // bytes between consecutive indices of dim i
+    stride *= dims[i];
+  }
+  CUresult r = g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdims,
+                        strides, gbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1,
+                          uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
+                          bool swizzle128) {
+  const uint64_t dims[3] = {dim0, dim1, dim2};
+  const uint32_t box[3] = {box0, box1, box2};
+  return encode_tensor_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3, dims, box, swizzle128);
 }
 
 namespace {
@@ -134,7 +149,9 @@ struct StoreRows {
   const int32_t* slot_mapping;
 };
 
-pa_status decode_impl(const StoreRows* store, void* out, const void* q, const void* k_cache,
+// k_scales / v_scales: non-null for e4m3 pools (pa_decode_fp8)
+pa_status decode_impl(const StoreRows* store, const float* k_scales, const float* v_scales,
+                      void* out, const void* q, const void* k_cache,
                       const void* v_cache, pa_cache_desc cache, const int32_t* block_tables,
                       int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
                       int32_t num_q_heads, float scale, int32_t max_context_len,
@@ -159,6 +176,9 @@ pa_status decode_impl(const StoreRows* store, void* out, const void* q, const vo
     return PA_ERR_INVALID_ARG;
   if (store && (!store->new_k || !store->new_v || !store->slot_mapping ||
                 !aligned16(store->new_k) || !aligned16(store->new_v)))
+    return PA_ERR_INVALID_ARG;
+  const bool fp8 = k_scales != nullptr || v_scales != nullptr;
+  if (fp8 && (!k_scales || !v_scales || !aligned16(k_scales) || !aligned16(v_scales)))
     return PA_ERR_INVALID_ARG;
   if (partition_size < 0 || (partition_size % 64) != 0) return PA_ERR_INVALID_ARG;
   const int P = partition_size > 0 ? partition_size
@@ -198,6 +218,13 @@ pa_status decode_impl(const StoreRows* store, void* out, const void* q, const vo
     a.new_k = store->new_k;
     a.new_v = store->new_v;
     a.slot_mapping = store->slot_mapping;
+  }
+  if (fp8) {
+    // e4m3 pools have only the tensor-core path
+    a.fp8 = true;
+    a.k_scales = k_scales;
+    a.v_scales = v_scales;
+    if (!decode_tc_supported(a)) return PA_ERR_UNSUPPORTED;
   }
   // the persistent kernel stores the new rows itself; the CUDA-core path stores them
   // with a checked kernel first
@@ -328,7 +355,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
                     float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
                     size_t workspace_bytes, void* stream) {
-  return decode_impl(nullptr, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+  return decode_impl(nullptr, nullptr, nullptr, out, q, k_cache, v_cache, cache, block_tables,
+                     max_blocks_per_seq,
                      context_lens, num_seqs, num_q_heads, scale, max_context_len, partition_size,
                      workspace, workspace_bytes, stream);
 }
@@ -341,9 +369,40 @@ pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* s
                           int32_t max_context_len, int32_t partition_size, void* workspace,
                           size_t workspace_bytes, void* stream) {
   const StoreRows rows{new_k, new_v, slot_mapping};
-  return decode_impl(&rows, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+  return decode_impl(&rows, nullptr, nullptr, out, q, k_cache, v_cache, cache, block_tables,
+                     max_blocks_per_seq,
                      context_lens, num_seqs, num_q_heads, scale, max_context_len, partition_size,
                      workspace, workspace_bytes, stream);
+}
+
+pa_status pa_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void* v_codes,
+                               float* k_scales, float* v_scales, pa_cache_desc cache,
+                               const int32_t* slot_mapping, int32_t num_tokens, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_codes || !v_codes || !k_scales || !v_scales || !slot_mapping)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes) ||
+      !aligned16(k_scales) || !aligned16(v_scales))
+    return PA_ERR_INVALID_ARG;
+  return finish(launch_store_kvcache_fp8(k, v, k_codes, v_codes, k_scales, v_scales, cache,
+                                         slot_mapping, num_tokens,
+                                         static_cast<cudaStream_t>(stream)),
+                stream);
+}
+
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_codes, const void* v_codes,
+                        const float* k_scales, const float* v_scales, pa_cache_desc cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                        float scale, int32_t max_context_len, int32_t partition_size,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k_scales || !v_scales) return PA_ERR_INVALID_ARG;
+  return decode_impl(nullptr, k_scales, v_scales, out, q, k_codes, v_codes, cache, block_tables,
+                     max_blocks_per_seq, context_lens, num_seqs, num_q_heads, scale,
+                     max_context_len, partition_size, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,

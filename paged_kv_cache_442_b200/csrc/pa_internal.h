@@ -26,6 +26,10 @@ cudaError_t ensure_max_dynamic_smem(const void* func, int bytes);
 
 // Encode a 3-D bf16 tensor map over a [dim2][dim1][dim0] row-major tensor.
 // swizzle128: 128-byte swizzle (box_dim0 * 2 must then be <= 128).
+// Any rank (<= 5), element type and size; dims innermost first; strides from dims.
+bool encode_tensor_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                       int elem_bytes, int rank, const uint64_t* dims, const uint32_t* box,
+                       bool swizzle128);
 bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1,
                           uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2,
                           bool swizzle128);
@@ -33,6 +37,10 @@ bool encode_tensor_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uin
 cudaError_t launch_block_hashes(const int32_t* token_ids, const int32_t* cu_tokens,
                                 const int32_t* cu_blocks, int32_t num_seqs, int32_t block_size,
                                 uint32_t* hashes_out, cudaStream_t stream);
+cudaError_t launch_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void* v_codes,
+                                     float* k_scales, float* v_scales, const pa_cache_desc& c,
+                                     const int32_t* slot_mapping, int32_t num_tokens,
+                                     cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const pa_cache_desc& c,
                                const int32_t* src_blocks, const int32_t* dst_blocks,
                                int32_t num_pairs, cudaStream_t stream);
@@ -62,6 +70,10 @@ struct DecodeLaunch {
   const void* new_k = nullptr;
   const void* new_v = nullptr;
   const int32_t* slot_mapping = nullptr;
+  // pa_decode_fp8: k_cache / v_cache hold e4m3 codes; scales [Hkv][num_blocks * bs] fp32
+  bool fp8 = false;
+  const float* k_scales = nullptr;
+  const float* v_scales = nullptr;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // Stores the new rows of a pa_store_decode call on its own (the paths whose decode

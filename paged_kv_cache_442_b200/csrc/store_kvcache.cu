@@ -6,6 +6,9 @@
 // consecutive threads take consecutive vectors of a row, so both the reads of
 // k/v and the writes into the pool row are fully coalesced. K and V are handled
 // by the same thread (two independent 16-byte transfers in flight).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
 #include "pa_internal.h"
 #include "pa_ptx.cuh"
 
@@ -68,7 +71,87 @@ __global__ void __launch_bounds__(128) store_last_rows_kernel(
   }
 }
 
+// fp8 pools: one warp per (token, kv head, K or V) row. The row's largest magnitude
+// sets its scale (amax / 448, fp32); codes are e4m3(x * (448 / amax)) rounded to
+// nearest even and saturated. A row whose 448 / amax is not a finite fp32 (all
+// zeros, or amax below 448 / FLT_MAX) stores zero codes and scale 0.
+template <int D>
+__global__ void __launch_bounds__(256) store_kvcache_fp8_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    uint8_t* __restrict__ k_codes, uint8_t* __restrict__ v_codes, float* __restrict__ k_scales,
+    float* __restrict__ v_scales, const int32_t* __restrict__ slot_mapping, int32_t num_tokens,
+    int32_t hkv, int64_t num_slots, unsigned* err) {
+  constexpr int PER = D / 32;  // values per lane
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t total = static_cast<int64_t>(num_tokens) * hkv * 2;
+  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < total;
+       w += warps) {
+    const int64_t t = w / (2 * hkv);
+    const int rem = static_cast<int>(w - t * 2 * hkv);
+    const int g = rem >> 1;
+    const bool is_v = rem & 1;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (lane == 0) flag_error(err, PA_DEV_ERR_BAD_INDEX);
+      continue;
+    }
+    const __nv_bfloat16* src = (is_v ? v : k) + (t * hkv + g) * D + lane * PER;
+    float x[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) x[i] = __bfloat162float(src[i]);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float inv = __fdiv_rn(448.f, amax);
+    const bool zero_row = isinf(inv);
+    if (zero_row) inv = 0.f;
+    // a zero row stores +0 codes (x * 0 would give -0 for negative x)
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < PER && !zero_row; i += 2) {
+      const __nv_fp8x2_storage_t two = __nv_cvt_float2_to_fp8x2(
+          make_float2(__fmul_rn(x[i], inv), __fmul_rn(x[i + 1], inv)), __NV_SATFINITE, __NV_E4M3);
+      packed |= static_cast<uint32_t>(two) << (8 * i);
+    }
+    uint8_t* dst = (is_v ? v_codes : k_codes) + (slot * hkv + g) * D + lane * PER;
+    if (PER == 4) {
+      *reinterpret_cast<uint32_t*>(dst) = packed;
+    } else {
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+    }
+    if (lane == 0)
+      (is_v ? v_scales : k_scales)[g * num_slots + slot] = zero_row ? 0.f : __fdiv_rn(amax, 448.f);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void* v_codes,
+                                     float* k_scales, float* v_scales, const pa_cache_desc& c,
+                                     const int32_t* slot_mapping, int32_t num_tokens,
+                                     cudaStream_t stream) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int64_t rows = static_cast<int64_t>(num_tokens) * c.num_kv_heads * 2;
+  int64_t blocks = (rows * 32 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  const int64_t num_slots = static_cast<int64_t>(c.num_blocks) * c.block_size;
+  if (c.head_dim == 128)
+    store_kvcache_fp8_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<uint8_t*>(k_codes), static_cast<uint8_t*>(v_codes), k_scales, v_scales,
+        slot_mapping, num_tokens, c.num_kv_heads, num_slots, device_error_word());
+  else
+    store_kvcache_fp8_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<uint8_t*>(k_codes), static_cast<uint8_t*>(v_codes), k_scales, v_scales,
+        slot_mapping, num_tokens, c.num_kv_heads, num_slots, device_error_word());
+  return cudaGetLastError();
+}
 
 cudaError_t launch_store_last_rows(const DecodeLaunch& a, cudaStream_t stream) {
   if (a.num_seqs == 0 || !a.slot_mapping) return cudaSuccess;

@@ -23,7 +23,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree():
@@ -160,3 +160,43 @@ def test_copy_blocks_argument_checks(lib):
     assert lib.pa_copy_blocks(FAKE, FAKE, d, NULL, FAKE, 2, NULL) == 1
     assert lib.pa_copy_blocks(FAKE, FAKE, desc(bs=12), FAKE, FAKE, 2, NULL) == 1
     assert lib.pa_copy_blocks(NULL, NULL, d, NULL, NULL, 0, NULL) == 0   # no-op
+
+
+def test_fp8_store_argument_checks(lib):
+    d = desc()
+    misaligned = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.pa_store_kvcache_fp8(FAKE, FAKE, FAKE, FAKE, NULL, FAKE, d, FAKE, 4, NULL) == 1
+    assert lib.pa_store_kvcache_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, misaligned, d, FAKE, 4, NULL) == 1
+    assert lib.pa_store_kvcache_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, desc(d=96), FAKE, 4, NULL) == 1
+    assert lib.pa_store_kvcache_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, -1, NULL) == 1
+    assert lib.pa_store_kvcache_fp8(NULL, NULL, NULL, NULL, NULL, NULL, d, NULL, 0, NULL) == 0
+
+
+def test_fp8_decode_argument_checks(lib):
+    ws = FAKE
+    d = desc(hkv=2)
+    # both scale arrays are required
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, NULL, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 32, 128,
+                             ws, 1 << 20, NULL) == 1
+    # only the tensor-core path reads e4m3 pools: 16 query heads per kv head, head dim
+    # 64 and partitions that are not a multiple of 128 are valid but not implemented
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 32, 0.1, 32, 128,
+                             ws, 1 << 20, NULL) == 2
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, desc(hkv=2, d=64), FAKE, 4, FAKE, 2, 4,
+                             0.1, 32, 128, ws, 1 << 20, NULL) == 2
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 32, 192,
+                             ws, 1 << 20, NULL) == 2
+    # the decode checks still apply: Hq not a multiple of Hkv
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 3, 0.1, 32, 128,
+                             ws, 1 << 20, NULL) == 1
+    assert lib.pa_decode_fp8(NULL, NULL, NULL, NULL, FAKE, FAKE, d, NULL, 4, NULL, 0, 4, 0.1, 32, 0,
+                             NULL, 0, NULL) == 0
+
+
+def test_binding_fp8_checks_pool_shapes():
+    import torch
+    k = torch.zeros(4, 2, 128, dtype=torch.bfloat16)
+    codes = torch.zeros(16, 16, 2, 128, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_store_kvcache_fp8(k, k, codes, codes, torch.zeros(2, 256), torch.zeros(2, 256),
+                                torch.zeros(4, dtype=torch.int32))

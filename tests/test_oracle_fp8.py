@@ -63,6 +63,26 @@ def test_quantize_rows_scale_amax_and_error_bound():
     assert np.all(zero_codes == 0) and np.all(zero_scales == 0)
 
 
+def test_quantize_rows_at_the_fp32_overflow_edge():
+    """448 / amax overflows fp32 below amax = 448 / FLT_MAX (~1.3166e-36): such rows
+    store zeros; just above it the row quantises normally, its scale an fp32
+    subnormal, and reads back within the error bound."""
+    flt_max = float(np.finfo(np.float32).max)
+    edge = 448.0 / flt_max
+    tiny = f32_to_bf16_bits(np.array([[0.5 * edge, -0.25 * edge, 0.0, 1e-40]], np.float32))
+    codes, scales = fp8.quantize_rows(tiny)
+    assert np.all(codes == 0) and np.all(scales == 0)
+    row = np.array([[2.0 * edge, -edge, 0.5 * edge, 0.0]], np.float32)
+    bits = f32_to_bf16_bits(row)
+    codes, scales = fp8.quantize_rows(bits)
+    xf = oracle.bf16_bits_to_f64(bits)
+    assert codes[0, 0] == 0x7E and codes[0, 3] == 0
+    assert 0 < scales[0] < np.finfo(np.float32).tiny          # subnormal fp32 scale
+    assert abs(float(scales[0]) - np.max(np.abs(xf)) / 448.0) <= 2.0 ** -149
+    err = np.abs(fp8.dequantize(codes, scales) - xf)
+    assert np.all(err <= 2.0 ** -4 * np.abs(xf) + 2.0 ** -149 * 448)
+
+
 def test_decode_of_exactly_representable_rows_equals_bf16_decode():
     """Rows whose values are e4m3 values times a power of two scale survive quantising
     exactly, so the fp8 decode must equal the bf16 decode of the same rows."""
