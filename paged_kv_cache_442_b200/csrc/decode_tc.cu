@@ -41,13 +41,13 @@
 // fp8 variant (pa_decode_fp8): the pools hold e4m3 codes with one fp32 scale per
 // (position, kv head) row. The producer loads a tile's codes into the upper half of
 // its 32 KB ring slot and the tile's scales (one box per block, each on a 128-byte
-// boundary) into the lower half; warps 11-14 (converters) dequantise it in place:
-// thread r reads its row's 128 codes and its scale into registers, the 128 converter
-// threads meet at a named barrier (the scales sit where the first rows of the lower
-// half are written), and thread r writes its row as
-// bf16 (code * scale, rounded once) into both swizzled halves -- the upper-half write
-// covers exactly its own source row. The score, softmax, value and merge stages are
-// the bf16 ones, unchanged.
+// boundary) into a small area of the slot's own; converter warps (11-18 for up to 4
+// query heads per kv head, two threads per row; 11-14 for 8, one thread per row)
+// dequantise it in place: one of them waits for the bytes while the rest sleep in a
+// named barrier, each thread reads its share of a row's 128 codes and the row's scale
+// into registers, and after a warp sync (a row's upper-half bf16 covers only its own
+// codes) writes the row as bf16 (code * scale, rounded once) into both swizzled
+// halves. The score, softmax, value and merge stages are the bf16 ones, unchanged.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -73,8 +73,13 @@ constexpr int QS = 2;          // scheduler queue depth: one item prepared ahead
                                // queues reserve work early and unbalance the tail)
 constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flight)
 constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
-constexpr int kThreadsF8 = 480;  // + converters 11-14 (fp8 pools)
-constexpr int kConvWarp0 = 11;
+constexpr int kConvWarp0 = 11;   // fp8 pools: converter warps follow the scheduler
+// fp8: 8 converter warps (two threads per row of a tile) where the other roles fit in
+// the registers that leaves (608 threads: up to 4 query heads per kv head), else 4
+template <int G>
+constexpr int conv_warps() { return G <= 4 ? 8 : 4; }
+template <int G, bool F8>
+constexpr int tc_threads() { return kThreads + (F8 ? 32 * conv_warps<G>() : 0); }
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more than this
 constexpr int kRegion = TM * 128;            // 64 head dims x 128 positions (16 KB)
 constexpr int kTileBytes = 2 * kRegion;      // one K or V tile (32 KB)
@@ -102,6 +107,13 @@ constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
 constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS + NK + NV;
 constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+// fp8 only: each K / V ring slot's row scales are staged in a 1 KB area of their own
+// (one 128-byte-aligned box per block; block size >= 16 gives at most 8 boxes), so
+// converting a slot in place never overwrites scales another thread still has to read
+constexpr int kSclBytes = 1024;
+constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
+constexpr int kSmemBytesF8 = kOffScl + (NK + NV) * kSclBytes + 1024;
+static_assert(kSmemBytesF8 <= 227 * 1024, "shared memory per CTA (fp8)");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
               "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
 static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "tile sizes");
@@ -260,34 +272,25 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// two fp32 products in one instruction (sm_100 packed fp32), each rounded to nearest
-__device__ __forceinline__ float2 mul_f32x2(float2 a, float s) {
-  uint64_t r;
-  asm("{\n\t.reg .b64 ra, rb;\n\t"
-      "mov.b64 ra, {%1, %2};\n\t"
-      "mov.b64 rb, {%3, %3};\n\t"
-      "mul.rn.f32x2 %0, ra, rb;\n\t}"
-      : "=l"(r)
-      : "f"(a.x), "f"(a.y), "f"(s));
-  float2 o;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
-  return o;
-}
-
 // 16 e4m3 codes (one uint4, code i in byte i) times a scale -> 16 bf16 values as two
 // uint4 (values 0-7, 8-15; element i in the low half of word i/2 ... as bf16 pairs).
 // e4m3 -> f16 is exact, so code * scale is rounded once (fp32 product, then to bf16).
-__device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint4& lo, uint4& hi) {
+// Each step runs over all eight pairs before the next, so the eight chains overlap.
+__device__ __forceinline__ void dequant16(const uint4 raw, float2 scale2, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  __half2_raw h[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    h[i] = __nv_cvt_fp8x2_to_halfraw2(
+        static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu), __NV_E4M3);
+  float2 f[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __fmul2_rn(f[i], scale2);
   uint32_t out[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const __nv_fp8x2_storage_t two =
-        static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
-    const float2 f = mul_f32x2(__half22float2(*reinterpret_cast<const __half2*>(&h)), scale);
-    out[i] = pack_bf16x2(f.x, f.y);
-  }
+  for (int i = 0; i < 8; ++i) out[i] = pack_bf16x2(f[i].x, f[i].y);
   lo = make_uint4(out[0], out[1], out[2], out[3]);
   hi = make_uint4(out[4], out[5], out[6], out[7]);
 }
@@ -306,7 +309,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 
 template <int G, bool F8>
-__global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kernel(
+__global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmSK,
     const __grid_constant__ CUtensorMap tmSV, const TcParams p) {
@@ -354,15 +357,15 @@ __global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kerne
     reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
-    // fp8: a ring slot is full once the four converter warps have written it
+    // fp8: a ring slot is full once every converter warp has written its rows
     for (int i = 0; i < NK; ++i) {
-      mbar_init(&k_full[i], F8 ? 4 : 1);
+      mbar_init(&k_full[i], F8 ? conv_warps<G>() : 1);
       mbar_init(&k_empty[i], 1);
       mbar_init(&kst_full[i], 1);
       conv_stop[i] = 0;
     }
     for (int i = 0; i < NV; ++i) {
-      mbar_init(&v_full[i], F8 ? 4 : 1);
+      mbar_init(&v_full[i], F8 ? conv_warps<G>() : 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&vst_full[i], 1);
     }
@@ -494,14 +497,15 @@ __global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kerne
         if (lane == 0) {
           uint8_t* kdst = smem + kOffK + ks * kTileBytes;
           if (F8) {
-            // codes into the upper half of the slot, scales into its first 512 bytes
+            // codes into the upper half of the slot, scales into the slot's scale area
             mbar_arrive_expect_tx(&kst_full[ks], kRegion + TM * 4);
             for (int b = 0; b < nbox; ++b) {
               const int pos = t0 + i * TM + b * rows;
               const int bi = (pos >> p.bs_log2) - first_blk;
               const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
               tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &kst_full[ks], 0, g, row);
-              tma_load_2d(kdst + b * sstride, &tmSK, &kst_full[ks], row, g);
+              tma_load_2d(smem + kOffScl + ks * kSclBytes + b * sstride, &tmSK, &kst_full[ks],
+                          row, g);
             }
           } else {
             mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
@@ -530,7 +534,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kerne
               const int bi = (pos >> p.bs_log2) - first_blk;
               const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
               tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &vst_full[vs], 0, g, row);
-              tma_load_2d(vdst + b * sstride, &tmSV, &vst_full[vs], row, g);
+              tma_load_2d(smem + kOffScl + (NK + vs) * kSclBytes + b * sstride, &tmSV,
+                          &vst_full[vs], row, g);
             }
           } else {
             mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
@@ -927,45 +932,60 @@ __global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kerne
       ++k;
     }
   } else if (F8) {
-    // ======================================================== converter warps 11-14
-    // Follow the tile sequence of the producer; thread r dequantises row r of each K
-    // and V tile in place. Every thread waits on its own; the barrier vote that follows
-    // both lets them leave together and keeps every write behind every read of the
-    // slot's scales (which lie where the first rows of the lower half are written).
-    const int r = tid - kConvWarp0 * 32;
+    // ======================================================== converter warps 11..
+    // Follow the tile sequence of the producer; PPR threads (adjacent lanes) share row
+    // r of each K and V tile and dequantise it in place, CPT 16-byte chunks of codes
+    // each. One thread polls the staging barrier while the others sleep in a named
+    // barrier (spinning warps would take issue slots from the MMA and TMA threads);
+    // the vote there also carries abort and end-of-tiles. A row's upper-half bf16
+    // covers only that row's codes, so a warp-level sync orders reads before writes.
+    constexpr int NCT = 32 * conv_warps<G>();
+    constexpr int PPR = NCT / TM;
+    constexpr int CPT = 8 / PPR;
+    const int t = tid - kConvWarp0 * 32;
+    const int r = t / PPR;
+    const int part = t % PPR;
     const int sw = r & 7;
+    const int rot = r & (CPT - 1);
     // where the producer put row r's scale: box r / rows, 128-byte aligned boxes
     const int rows = bs < TM ? bs : TM;
     const int soff = (r / rows) * (rows * 4 < 128 ? 128 : rows * 4) + (r % rows) * 4;
     // stop_slot: the K ring slot whose end-of-tiles mark to honour, or -1 (V tiles)
-    auto convert = [&](uint8_t* slot, uint64_t* staged, unsigned parity, uint64_t* full,
-                       int stop_slot) -> bool {
-      bool ok = wait_or_abort(staged, parity, p.err, abort_flag);
-      const bool stop = ok && stop_slot >= 0 && conv_stop[stop_slot] != 0;
-      uint4 raw[8];
-      float sc = 0.f;
-      if (ok && !stop) {
-        // chunk c ^ (r % 8) of the row in step c: the 8 threads of a quarter warp read
-        // 8 different 16-byte bank groups (rows are 128 bytes apart)
-        const uint4* src = reinterpret_cast<const uint4*>(slot + kRegion + r * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) raw[c] = src[c ^ sw];
-        sc = *reinterpret_cast<const float*>(slot + soff);
+    auto convert = [&](uint8_t* slot, const uint8_t* scl, uint64_t* staged, unsigned parity,
+                       uint64_t* full, int stop_slot) -> bool {
+      bool quit = false;
+      if (t == 0) {
+        quit = !wait_or_abort(staged, parity, p.err, abort_flag) ||
+               (stop_slot >= 0 && conv_stop[stop_slot] != 0);
       }
-      if (bar_or(3, 128, !ok || stop)) return false;
+      if (bar_or(3, NCT, quit)) return false;
+      // the phase is complete (the slot cannot refill before this tile is consumed):
+      // each thread's own test of it orders the TMA's bytes before its reads
+      if (!mbar_try_wait(staged, parity)) flag_error(p.err, PA_DEV_ERR_TIMEOUT);
+      uint4 raw[CPT];
+      // code chunk part * CPT + (c ^ rot) of the row in step c: the 8 threads of a
+      // quarter warp read 8 different 16-byte bank groups (rows are 128 bytes apart)
+      const uint4* src = reinterpret_cast<const uint4*>(slot + kRegion + r * 128);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < CPT; ++c) raw[c] = src[part * CPT + (c ^ rot)];
+      const float scv = *reinterpret_cast<const float*>(scl + soff);
+      const float2 sc2 = make_float2(scv, scv);
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
         uint4 lo, hi;
-        dequant16(raw[c], sc, lo, hi);
-        // dims 16k..16k+15 (k = c ^ (r % 8)) = 16-byte bf16 chunks 2k and 2k+1 of the
-        // row; chunk q lies in half q / 8 at position (q % 8) ^ (r % 8) (128-byte
-        // swizzle). For each (c, h) the quarter warp's 8 positions are distinct.
+        dequant16(raw[c], sc2, lo, hi);
+        // dims 16k..16k+15 = 16-byte bf16 chunks 2k (lo) and 2k+1 (hi) of the row;
+        // chunk q lies in half q / 8 at position (q % 8) ^ (r % 8) (128-byte swizzle).
+        // The two threads of a row write their chunk pairs in opposite orders, so for
+        // every step the quarter warp's 8 positions are distinct.
+        const int kc = part * CPT + (c ^ rot);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int q = 2 * (c ^ sw) + h;
+          const int q = 2 * kc + (h ^ (PPR == 2 ? part : 0));
           uint4* dst = reinterpret_cast<uint4*>(slot + (q >> 3) * kRegion + r * 128 +
                                                 (((q & 7) ^ sw) << 4));
-          *dst = h ? hi : lo;
+          *dst = (q & 1) ? hi : lo;
         }
       }
       fence_proxy_async_smem();
@@ -973,12 +993,18 @@ __global__ void __launch_bounds__(F8 ? kThreadsF8 : kThreads, 1) decode_tc_kerne
       if (lane == 0) mbar_arrive(full);
       return true;
     };
-    for (unsigned j = 0;; ++j) {
-      const int ks = j % NK;
-      if (!convert(smem + kOffK + ks * kTileBytes, &kst_full[ks], (j / NK) & 1, &k_full[ks], ks))
-        break;
-      const int vs = j % NV;
-      if (!convert(smem + kOffV + vs * kTileBytes, &vst_full[vs], (j / NV) & 1, &v_full[vs], -1))
+    // K(0), V(0), K(1), ... through one call site (keeps the unrolled conversion's
+    // code once in the instruction cache)
+#pragma unroll 1
+    for (unsigned i = 0;; ++i) {
+      const unsigned j = i >> 1;
+      const bool is_v = i & 1;
+      const int rs = is_v ? j % NV : j % NK;
+      const unsigned ph = is_v ? (j / NV) & 1 : (j / NK) & 1;
+      uint8_t* slot = smem + (is_v ? kOffV : kOffK) + rs * kTileBytes;
+      const uint8_t* scl = smem + kOffScl + (is_v ? NK + rs : rs) * kSclBytes;
+      if (!convert(slot, scl, is_v ? &vst_full[rs] : &kst_full[rs], ph,
+                   is_v ? &v_full[rs] : &k_full[rs], is_v ? -1 : rs))
         break;
     }
   }
@@ -1033,13 +1059,14 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
     tmSK = tmQ;  // unused by the bf16 kernel
     tmSV = tmQ;
   }
+  constexpr int smem_bytes = F8 ? kSmemBytesF8 : kSmemBytes;
   cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<G, F8>),
-                                          kSmemBytes);
+                                          smem_bytes);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  decode_tc_kernel<G, F8><<<grid, F8 ? kThreadsF8 : kThreads, kSmemBytes, stream>>>(
+  decode_tc_kernel<G, F8><<<grid, tc_threads<G, F8>(), smem_bytes, stream>>>(
       tmQ, tmK, tmV, tmSK, tmSV, p);
   return cudaGetLastError();
 }
@@ -1048,7 +1075,7 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
 
 bool decode_tc_supported(const DecodeLaunch& a) {
   const int G = a.num_q_heads / a.cache.num_kv_heads;
-  // fp8 pools add four converter warps (480 threads): up to 8 query heads per kv head
+  // fp8 pools add four or eight converter warps: up to 8 query heads per kv head
   const bool g_ok = a.fp8 ? (G == 1 || G == 2 || G == 4 || G == 8)
                           : (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
   // fp8 scale boxes start at slot index (block id * block size): a multiple of four
