@@ -482,9 +482,13 @@ def main():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--separate-store", action="store_true",
                     help="decode steps as pa_store_kvcache + pa_decode instead of pa_store_decode")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="print only the decode-batch-64 step over e4m3 pools (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.fp8_only and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        ap.error("--fp8-only runs on one GPU")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -513,6 +517,12 @@ def main():
             pg.barrier()
 
     hbm_peak, tf_peak, tf_sustained, peak_src = peaks()
+    if args.fp8_only:
+        if rank == 0:
+            print(json.dumps({"decode_b64_fp8": measure_fp8_decode(
+                torch, pa, hbm_peak, peak_src, None, steps=args.steps, warmup=args.warmup)}),
+                flush=True)
+        return
     # every rank decodes its own batch of the same shape (weak scaling)
     w = rank_workload(cfg, rank)
     runner = GpuRunner(w, torch, pa, args.partition_size, args.separate_store)
