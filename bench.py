@@ -375,6 +375,60 @@ def time_steps(runner, torch, steps, warmup, flush_buf, barrier=None):
     return sum(step_ms), attn_ms, launches // steps
 
 
+def decode_counter_bytes(w):
+    """The leading block of the decode workspace that holds the tagged work and arrival
+    counters (include/pa.h, pa_decode_workspace_size)."""
+    return -(-(8 * (1 + w.num_seqs * w.num_q_heads)) // 256) * 256
+
+
+def time_graph(runner, torch, steps, warmup, flush_buf):
+    """The decode step replayed from a CUDA graph (launch overhead out of the picture).
+
+    A captured call keeps the counter tag it was captured with, so the graph first
+    clears the workspace's counter block (a replay is then a fresh call). Returns
+    (mean step us, whether the replayed output equals the eager output bit for bit),
+    or an error string."""
+    try:
+        w = runner.w
+        n = decode_counter_bytes(w) // 4
+        runner.step()
+        torch.cuda.synchronize()
+        eager = runner.out.clone()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                runner.ws[:n].zero_()
+                runner.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            runner.ws[:n].zero_()
+            runner.step()
+        runner.out.zero_()
+        flush_out = torch.zeros((), dtype=flush_buf.dtype, device=flush_buf.device)
+        for _ in range(warmup):
+            torch.sum(flush_buf, dim=0, out=flush_out)
+            g.replay()
+        torch.cuda.synchronize()
+        same = bool(torch.equal(runner.out.view(torch.int16), eager.view(torch.int16)))
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            torch.sum(flush_buf, dim=0, out=flush_out)
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        us = sum(a.elapsed_time(b) for a, b in ev) / steps * 1e3
+        del g
+        return round(us, 2), same
+    except Exception as e:  # noqa: BLE001  (reported, not fatal to the run)
+        return None, f"{type(e).__name__}: {e}"
+
+
 def time_e2e(runner, torch, steps, warmup):
     """Same step through the host: pinned host inputs copied in, output copied out."""
     w = runner.w
@@ -453,11 +507,11 @@ def host_threads():
     return cores, blas
 
 
-def cpu_oracle_time(w, budget_s=12.0):
+def cpu_oracle_time(w, budget_s=12.0, pools=None):
     """The oracle (as it stands) decoding sequences one at a time for ~budget_s.
 
     Returns (seconds, bytes, sequences decoded, cores, blas threads)."""
-    pools = oracle_pools_for(w)
+    pools = oracle_pools_for(w) if pools is None else pools
     tot_t, tot_b, n = 0.0, 0, 0
     while tot_t < budget_s:
         dt, nb = oracle_decode_one(w, pools, n % w.num_seqs)
@@ -466,6 +520,17 @@ def cpu_oracle_time(w, budget_s=12.0):
         n += 1
     cores, blas = host_threads()
     return tot_t, tot_b, n, cores, blas
+
+
+def cpu_oracle_time_one_core(w, budget_s=4.0):
+    """The same oracle with its BLAS limited to one thread (GB/s, sequences decoded)."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # noqa: BLE001
+        return None, 0
+    with threadpool_limits(limits=1):
+        t, b, n, _, _ = cpu_oracle_time(w, budget_s)
+    return b / t / 1e9, n
 
 
 # --------------------------------------------------------------------------- main
@@ -566,6 +631,12 @@ def main():
                     "traffic": recorded_traffic(cfg.name + ".prefill", PREFILL_SRC)}
 
     e2e_ms, h2d, d2h = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
+    graph = None
+    if w.kind == "decode" and not args.headline_only:
+        g_us, g_same = time_graph(runner, torch, min(args.steps, 500), args.warmup, flush)
+        graph = {"step_us": g_us, "eager_step_us": round(step_ms * 1e3, 2),
+                 "output_equals_eager": g_same,
+                 "graph": "clear the workspace counter block, then the step's library call"}
     e2e_step_ms = max_over_ranks(e2e_ms / min(args.steps, 500), pg, torch, "cuda")
 
     line = {
@@ -600,6 +671,7 @@ def main():
                         "paged_kv_cache_442_b200.pa_store_kvcache + pa_decode") +
                        " (C ABI) on pinned host buffers"},
         "gpu_launches": launches_per_step * args.steps,
+        "cuda_graph": graph,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.headline_only:
@@ -614,6 +686,10 @@ def main():
                                 "blas_threads": blas, "kind": "oracle",
                                 "sample": f"oracle decode of {n} single sequences of {cfg.name} "
                                           f"on its own pools ({ct:.1f} s of CPU time)"}
+        v1, n1 = cpu_oracle_time_one_core(w)
+        if v1 is not None:
+            line["cpu_baseline"]["value_one_blas_thread"] = round(v1, 4)
+            line["cpu_baseline"]["sample_one_blas_thread"] = f"{n1} sequences, ~4 s"
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()

@@ -220,6 +220,14 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *                  not matter (its counters carry a tag unique to each call, so
  *                  leftovers of earlier calls never count). Calls that overlap
  *                  on the GPU must use different workspaces.
+ *                  CUDA graphs: the tag is drawn on the host when the call is
+ *                  made, so a captured call replays with its capture's tag. Clear
+ *                  the workspace's leading counter block (the 256-byte-rounded
+ *                  8 * (1 + num_seqs * num_q_heads) bytes) before each replay, e.g.
+ *                  with a memset node ahead of it in the same graph; a replay is
+ *                  then exactly a fresh call. The same holds for pa_store_decode
+ *                  and pa_decode_fp8. pa_decode_no_alloc's scratch belongs to the
+ *                  library and cannot be cleared by the caller: do not capture it.
  * Supported: Hq / Hkv in {1, 2, 4, 8} (and 16 when head_dim is 128).
  * head_dim 128 runs the persistent tcgen05 kernel (partition_size a multiple
  * of 128, at most 2048; other sizes run the CUDA-core kernel); head_dim 64 runs
