@@ -200,3 +200,16 @@ def test_binding_fp8_checks_pool_shapes():
     with pytest.raises(ValueError, match="CUDA"):
         pa.pa_store_kvcache_fp8(k, k, codes, codes, torch.zeros(2, 256), torch.zeros(2, 256),
                                 torch.zeros(4, dtype=torch.int32))
+
+
+def test_bench_counter_block_matches_the_library(lib):
+    """The graph-replay path clears the workspace's counter block; its size in the
+    benchmark must be the library's (the workspace size when nothing is split)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from workloads import CONFIGS, generate
+    w = generate(CONFIGS["tiny_decode"])
+    for B, Hq in ((w.num_seqs, w.num_q_heads), (64, 16), (512, 32), (1, 1)):
+        w.num_seqs, w.num_q_heads = B, Hq
+        assert bench.decode_counter_bytes(w) == pa.pa_decode_workspace_size(B, Hq, 128, 256, 256)
