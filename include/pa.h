@@ -121,6 +121,21 @@ void pa_bm_destroy(pa_block_manager* bm);
 pa_status pa_bm_allocate(pa_block_manager* bm, const int32_t* token_ids, int32_t num_tokens,
                          const uint32_t* block_hashes, int32_t* table_out);
 
+/* pa_bm_allocate for a batch of requests in one call, in order (a scheduler admitting
+ * a step's prefills). token_ids: the requests back to back; cu_tokens int32
+ * [num_seqs + 1] (cu_tokens[0] = 0) their offsets. block_hashes: NULL, or each
+ * request's full-block hashes back to back at offsets cu_blocks [num_seqs + 1]
+ * (cu_blocks[s+1] - cu_blocks[s] = length_s / block_size). tables_out: every request's
+ * table back to back, ceil(length_s / block_size) entries each. *num_done: the number
+ * of requests allocated. When the pool runs out at request s, the call returns
+ * PA_ERR_NO_BLOCKS with *num_done = s: requests 0..s-1 keep their blocks (free them,
+ * or run them), request s holds nothing. Bad offsets return PA_ERR_INVALID_ARG before
+ * any block is taken. */
+pa_status pa_bm_allocate_batch(pa_block_manager* bm, const int32_t* token_ids,
+                               const int32_t* cu_tokens, int32_t num_seqs,
+                               const uint32_t* block_hashes, const int32_t* cu_blocks,
+                               int32_t* tables_out, int32_t* num_done);
+
 /* A finished request: one reference dropped per entry; blocks reaching zero go back to
  * the free list. An id outside the pool or a block released more often than it is held
  * returns PA_ERR_INVALID_ARG and changes nothing. */

@@ -19,7 +19,8 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
                 4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT", 6: "PA_ERR_NO_BLOCKS"}
 
 # every extern "C" function include/pa.h declares
-EXPORTED = ("pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_free", "pa_bm_append",
+EXPORTED = ("pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_allocate_batch", "pa_bm_free",
+            "pa_bm_append",
             "pa_bm_num_used", "pa_bm_ref_counts", "pa_block_hashes",
             "pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
             "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill",
@@ -64,6 +65,8 @@ def load_library(path: str | None = None):
     lib.pa_bm_destroy.restype = None
     lib.pa_bm_allocate.argtypes = [vp, vp, i32, vp, vp]
     lib.pa_bm_allocate.restype = ctypes.c_int
+    lib.pa_bm_allocate_batch.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32p]
+    lib.pa_bm_allocate_batch.restype = ctypes.c_int
     lib.pa_bm_free.argtypes = [vp, vp, i32]
     lib.pa_bm_free.restype = ctypes.c_int
     lib.pa_bm_append.argtypes = [vp, vp, i32p, i32, i32, i32, i32p, i32p, i32p]
@@ -305,6 +308,38 @@ class BlockManager:
                                      hs.ctypes.data if hs is not None else None, table.ctypes.data)
         _raise("pa_bm_allocate", st)
         return table.tolist()
+
+    def allocate_batch(self, requests, block_hashes=None):
+        """Tables of several requests in one library call, in order. Returns (tables,
+        number allocated); when the pool runs out the status is raised after the
+        allocated prefix is recorded in the exception's `done` attribute."""
+        np = self._np
+        lens = np.array([len(r) for r in requests], dtype=np.int64)
+        cu = np.zeros(len(requests) + 1, dtype=np.int32)
+        cu[1:] = np.cumsum(lens)
+        toks = (np.concatenate([np.asarray(r, dtype=np.int32) for r in requests])
+                if len(requests) and cu[-1] else np.zeros(1, dtype=np.int32))
+        nblk = -(-lens // self.block_size)
+        out = np.zeros(max(1, int(nblk.sum())), dtype=np.int32)
+        hs = cub = None
+        if block_hashes is not None:
+            hs = np.concatenate([np.asarray(h, dtype=np.uint32) for h in block_hashes]
+                                + [np.zeros(1, np.uint32)])
+            cub = np.zeros(len(requests) + 1, dtype=np.int32)
+            cub[1:] = np.cumsum([len(h) for h in block_hashes])
+        done = ctypes.c_int32(0)
+        st = self.lib.pa_bm_allocate_batch(self.h, toks.ctypes.data, cu.ctypes.data, len(requests),
+                                           hs.ctypes.data if hs is not None else None,
+                                           cub.ctypes.data if cub is not None else None,
+                                           out.ctypes.data, ctypes.byref(done))
+        offs = np.concatenate([[0], np.cumsum(nblk)])
+        tables = [out[offs[i]:offs[i + 1]].tolist() for i in range(done.value)]
+        if st != PA_OK:
+            err = PAError("pa_bm_allocate_batch", st)
+            err.done = done.value
+            err.tables = tables
+            raise err
+        return tables
 
     def free(self, table) -> None:
         t = self._np.ascontiguousarray(table, dtype=self._np.int32)

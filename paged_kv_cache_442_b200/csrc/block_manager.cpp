@@ -199,6 +199,37 @@ pa_status pa_bm_allocate(pa_block_manager* m, const int32_t* token_ids, int32_t 
   return PA_OK;
 }
 
+pa_status pa_bm_allocate_batch(pa_block_manager* m, const int32_t* token_ids,
+                               const int32_t* cu_tokens, int32_t num_seqs,
+                               const uint32_t* block_hashes, const int32_t* cu_blocks,
+                               int32_t* tables_out, int32_t* num_done) {
+  if (!m || num_seqs < 0 || !num_done || (num_seqs > 0 && (!cu_tokens || !tables_out)))
+    return PA_ERR_INVALID_ARG;
+  *num_done = 0;
+  if (num_seqs == 0) return PA_OK;
+  if (cu_tokens[0] != 0) return PA_ERR_INVALID_ARG;
+  if (block_hashes && (!cu_blocks || cu_blocks[0] != 0)) return PA_ERR_INVALID_ARG;
+  const int32_t bs = m->bs;
+  // validate every request before taking any block
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int32_t len = cu_tokens[s + 1] - cu_tokens[s];
+    if (len < 0) return PA_ERR_INVALID_ARG;
+    if (len > 0 && !token_ids) return PA_ERR_INVALID_ARG;
+    if (block_hashes && cu_blocks[s + 1] - cu_blocks[s] != len / bs) return PA_ERR_INVALID_ARG;
+  }
+  int64_t off = 0;
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int32_t len = cu_tokens[s + 1] - cu_tokens[s];
+    const pa_status st = pa_bm_allocate(m, token_ids ? token_ids + cu_tokens[s] : nullptr, len,
+                                        block_hashes ? block_hashes + cu_blocks[s] : nullptr,
+                                        tables_out + off);
+    if (st != PA_OK) return st;  // requests before s stay allocated; s holds nothing
+    off += (len + bs - 1) / bs;
+    *num_done = s + 1;
+  }
+  return PA_OK;
+}
+
 pa_status pa_bm_free(pa_block_manager* m, const int32_t* table, int32_t num_entries) {
   if (!m || num_entries < 0 || (num_entries > 0 && !table)) return PA_ERR_INVALID_ARG;
   // validate first: every id in the pool and held at least as often as it is listed

@@ -137,3 +137,62 @@ def test_native_append_cases_match_fixture():
             r2 = nat.append(tn[op[1]], op[2], op[3])
             assert r1 == r2 and tp[op[1]] == tn[op[1]]
         assert np.array_equal(nat.ref_counts(), np.array(py.ref_counts()))
+
+
+@pytest.mark.parametrize("bs,seed", [(1, 11), (4, 12), (16, 13)])
+def test_batch_allocation_equals_one_call_per_request(bs, seed):
+    """pa_bm_allocate_batch gives the tables and reference counts of allocating the same
+    requests one call at a time, with and without precomputed block hashes."""
+    rng = np.random.default_rng(seed)
+    nb = 4096 // bs + 64
+    order = rng.permutation(nb)
+    prefixes = [rng.integers(1, 50, size=rng.integers(1, 40)).tolist() for _ in range(3)]
+    reqs = make_requests(rng, 120, prefixes)
+    one = pa.BlockManager(nb, bs, free_order=order)
+    want = [one.allocate(r) for r in reqs]
+    for hashes in (None, [oracle.block_hashes(r, bs) for r in reqs]):
+        batch = pa.BlockManager(nb, bs, free_order=order)
+        got = batch.allocate_batch(reqs, block_hashes=hashes)
+        assert got == want
+        assert np.array_equal(batch.ref_counts(), one.ref_counts())
+        # and the tables free cleanly
+        for t in got:
+            batch.free(t)
+        assert batch.num_used() == 0
+
+
+def test_batch_allocation_stops_at_the_first_request_that_does_not_fit():
+    bs = 4
+    reqs = [list(range(1, 9)), list(range(20, 33)), list(range(40, 60)), [7, 7]]
+    bm = pa.BlockManager(6, bs)           # 2 + 4 blocks fit, the third request does not
+    with pytest.raises(pa.PAError) as e:
+        bm.allocate_batch(reqs)
+    assert e.value.status == 6 and e.value.done == 2
+    assert [len(t) for t in e.value.tables] == [2, 4]
+    ref = pa.BlockManager(6, bs)
+    ref.allocate(reqs[0])
+    ref.allocate(reqs[1])
+    assert np.array_equal(bm.ref_counts(), ref.ref_counts())   # request 2 holds nothing
+
+
+def test_batch_allocation_argument_checks():
+    import ctypes
+    bm = pa.BlockManager(16, 4)
+    lib = pa.load_library()
+    toks = np.arange(1, 11, dtype=np.int32)
+    cu = np.array([0, 6, 10], dtype=np.int32)
+    out = np.zeros(8, dtype=np.int32)
+    done = ctypes.c_int32(-1)
+    # hash offsets that disagree with the lengths (6 tokens = 1 full block, not 2)
+    hs = np.zeros(3, dtype=np.uint32)
+    cub = np.array([0, 2, 3], dtype=np.int32)
+    st = lib.pa_bm_allocate_batch(bm.h, toks.ctypes.data, cu.ctypes.data, 2, hs.ctypes.data,
+                                  cub.ctypes.data, out.ctypes.data, ctypes.byref(done))
+    assert st == 1 and done.value == 0 and bm.num_used() == 0
+    bad_cu = np.array([1, 6, 10], dtype=np.int32)
+    st = lib.pa_bm_allocate_batch(bm.h, toks.ctypes.data, bad_cu.ctypes.data, 2, None, None,
+                                  out.ctypes.data, ctypes.byref(done))
+    assert st == 1 and bm.num_used() == 0
+    st = lib.pa_bm_allocate_batch(bm.h, toks.ctypes.data, cu.ctypes.data, 0, None, None,
+                                  out.ctypes.data, ctypes.byref(done))
+    assert st == 0 and done.value == 0
