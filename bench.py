@@ -429,48 +429,116 @@ def time_graph(runner, torch, steps, warmup, flush_buf):
         return None, f"{type(e).__name__}: {e}"
 
 
+class PackedInputs:
+    """One step's host inputs packed into a single pinned buffer (q, new K/V rows,
+    slots, context lengths, block tables; each piece on a 256-byte boundary) and a
+    device buffer of the same layout whose typed views the library call takes, so a
+    step's inputs cross PCIe in ONE host-to-device copy and its output in one
+    device-to-host copy."""
+
+    def __init__(self, runner, torch):
+        pieces = [("q", runner.q), ("k", runner.new_k), ("v", runner.new_v),
+                  ("slots", runner.new_slots), ("ctx", runner.context_lens),
+                  ("bt", runner.block_tables)]
+        self.layout, off = {}, 0
+        for name, t in pieces:
+            if t is None:
+                continue
+            n = t.numel() * t.element_size()
+            self.layout[name] = (off, n, t.dtype, tuple(t.shape))
+            off += -(-n // 256) * 256
+        self.nbytes = off
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for name, t in pieces:
+            if t is not None:
+                o, n, _, _ = self.layout[name]
+                self.host[o:o + n].copy_(t.contiguous().view(torch.uint8).view(-1).cpu())
+        self.torch = torch
+
+    def device_views(self, dev_buf):
+        views = {}
+        for name, (o, n, dt, shape) in self.layout.items():
+            views[name] = dev_buf[o:o + n].view(dt).view(shape)
+        return views
+
+
 def time_e2e(runner, torch, steps, warmup):
-    """Same step through the host: pinned host inputs copied in, output copied out."""
-    w = runner.w
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    h_q = pin(runner.q)
-    h_k = pin(runner.new_k) if runner.new_k is not None else None
-    h_v = pin(runner.new_v) if runner.new_v is not None else None
-    h_slots = pin(runner.new_slots)
-    h_ctx = pin(runner.context_lens)
-    h_bt = pin(runner.block_tables)
-    h_out = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
-    d_q, d_ctx, d_bt = torch.empty_like(runner.q), torch.empty_like(runner.context_lens), \
-        torch.empty_like(runner.block_tables)
-    d_k = torch.empty_like(runner.new_k) if h_k is not None else None
-    d_v = torch.empty_like(runner.new_v) if h_v is not None else None
-    d_slots = torch.empty_like(runner.new_slots)
+    """The step through the host, as a caller without device-resident inputs runs it:
+    every step copies its packed inputs from pinned host memory to the device (one
+    copy), makes the library call on them, and copies the output back (one copy), all
+    in order on one stream. Returns (total ms, h2d bytes, d2h bytes, pipelined ms):
+    the last is the same steps with two buffer sets, the copies on a second stream
+    overlapping the previous step's kernel (a serving loop's steady state)."""
+    pk = PackedInputs(runner, torch)
+    d_in = torch.empty(pk.nbytes, dtype=torch.uint8, device="cuda")
+    v = pk.device_views(d_in)
     d_out = torch.empty_like(runner.out)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_ctx, h_bt) if t is not None)
+    h_out = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+    h2d = pk.nbytes
     d2h = h_out.numel() * h_out.element_size()
 
-    def one():
-        d_q.copy_(h_q, non_blocking=True)
-        d_ctx.copy_(h_ctx, non_blocking=True)
-        d_bt.copy_(h_bt, non_blocking=True)
-        d_slots.copy_(h_slots, non_blocking=True)
-        if d_k is not None:
-            d_k.copy_(h_k, non_blocking=True)
-            d_v.copy_(h_v, non_blocking=True)
-            runner.store(d_k, d_v, d_slots)
-        runner.attend(d_q, d_ctx, d_bt, d_out, d_k, d_v, d_slots)
+    def one(views, dout, hout, copy_stream=None):
+        d = views
+        runner.store(d.get("k"), d.get("v"), d["slots"])
+        runner.attend(d["q"], d["ctx"], d["bt"], dout, d.get("k"), d.get("v"), d["slots"])
+
+    def serial():
+        d_in.copy_(pk.host, non_blocking=True)
+        one(v, d_out, h_out)
         h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(warmup):
-        one()
+        serial()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for _ in range(steps):
-        one()
+        serial()
     e.record()
     torch.cuda.synchronize()
-    return s.elapsed_time(e), h2d, d2h
+    serial_ms = s.elapsed_time(e)
+    if not torch.equal(h_out.view(torch.int16), runner.out.cpu().view(torch.int16)):
+        # the step is deterministic: the copied-back output must be the device one
+        raise RuntimeError("end-to-end output differs from the device-resident step")
+
+    # pipelined: buffer set i % 2; step i's input copy overlaps step i-1's kernel
+    main = torch.cuda.current_stream()
+    cs = torch.cuda.Stream()
+    bufs = [(torch.empty(pk.nbytes, dtype=torch.uint8, device="cuda"), torch.empty_like(runner.out),
+             torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()) for _ in range(2)]
+    views = [pk.device_views(b[0]) for b in bufs]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_k = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def pipelined(n):
+        for i in range(n):
+            b = i % 2
+            din, dout, hout = bufs[b]
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(ev_k[b])       # the kernel of step i-2 read this buffer
+                din.copy_(pk.host, non_blocking=True)
+                ev_in[b].record(cs)
+            main.wait_event(ev_in[b])
+            if i >= 2:
+                main.wait_event(ev_out[b])       # step i-2's output has been copied out
+            one(views[b], dout, hout)
+            ev_k[b].record(main)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_k[b])
+                hout.copy_(dout, non_blocking=True)
+                ev_out[b].record(cs)
+        main.wait_stream(cs)
+
+    pipelined(warmup)
+    torch.cuda.synchronize()
+    s.record(main)
+    cs.wait_event(s)
+    pipelined(steps)
+    e.record(main)
+    torch.cuda.synchronize()
+    return serial_ms, h2d, d2h, s.elapsed_time(e)
 
 
 # --------------------------------------------------------------------------- CPU (oracle) arm
@@ -630,7 +698,7 @@ def main():
                     "algorithmic_flops_per_launch": fl, "avg_launch_us": round(attn_avg_ms * 1e3, 2),
                     "traffic": recorded_traffic(cfg.name + ".prefill", PREFILL_SRC)}
 
-    e2e_ms, h2d, d2h = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
+    e2e_ms, h2d, d2h, e2e_pipe_ms = time_e2e(runner, torch, min(args.steps, 500), args.warmup)
     graph = None
     if w.kind == "decode" and not args.headline_only:
         g_us, g_same = time_graph(runner, torch, min(args.steps, 500), args.warmup, flush)
@@ -638,6 +706,7 @@ def main():
                  "output_equals_eager": g_same,
                  "graph": "clear the workspace counter block, then the step's library call"}
     e2e_step_ms = max_over_ranks(e2e_ms / min(args.steps, 500), pg, torch, "cuda")
+    e2e_pipe_step_ms = max_over_ranks(e2e_pipe_ms / min(args.steps, 500), pg, torch, "cuda")
 
     line = {
         "metric": METRIC,
@@ -669,7 +738,13 @@ def main():
                 "d2h_bytes_per_step": d2h,
                 "api": ("paged_kv_cache_442_b200.pa_store_decode" if runner.fused else
                         "paged_kv_cache_442_b200.pa_store_kvcache + pa_decode") +
-                       " (C ABI) on pinned host buffers"},
+                       " (C ABI) on pinned host buffers",
+                "copies_per_step": "one packed host-to-device copy of all inputs, one "
+                                   "device-to-host copy of the output, in order on one stream",
+                "pipelined": {"value": round(job_gbps(job_bytes, e2e_pipe_step_ms), 1),
+                              "ms_per_step": round(e2e_pipe_step_ms, 5),
+                              "how": "two buffer sets; each step's copies on a second stream "
+                                     "overlap the previous step's kernel"}},
         "gpu_launches": launches_per_step * args.steps,
         "cuda_graph": graph,
         "clocks": clocks,
@@ -690,6 +765,15 @@ def main():
         if v1 is not None:
             line["cpu_baseline"]["value_one_blas_thread"] = round(v1, 4)
             line["cpu_baseline"]["sample_one_blas_thread"] = f"{n1} sequences, ~4 s"
+            if not args.headline_only:
+                # the one-core oracle on the other decode configurations as well
+                one = {}
+                for name in ("tiny_decode", "long_ctx_decode"):
+                    wo = generate(CONFIGS[name])
+                    g1, k1 = cpu_oracle_time_one_core(wo)
+                    one[name] = {"GBps": round(g1, 4), "sample": f"{k1} sequences, ~4 s"}
+                    del wo
+                line["cpu_baseline"]["one_blas_thread_other_configs"] = one
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()

@@ -34,8 +34,10 @@
  * ------
  *  - Arguments are validated on the host before any launch; a bad argument
  *    returns PA_ERR_INVALID_ARG and launches nothing. Supported sizes:
- *    head_dim 64 or 128; block_size a power of two in [16, 1024];
- *    num_q_heads a multiple of num_kv_heads.
+ *    head_dim 64 or 128 for the store, copy and decode entry points, 128 only
+ *    for pa_prefill, pa_store_prefill and pa_decode_fp8 (other head dims
+ *    return PA_ERR_UNSUPPORTED there); block_size a power of two in
+ *    [16, 1024]; num_q_heads a multiple of num_kv_heads.
  *  - A valid but unimplemented combination returns PA_ERR_UNSUPPORTED.
  *  - A failed launch returns PA_ERR_CUDA.
  *  - Device-side index checks never trap: an out-of-range block id or slot is
@@ -129,8 +131,8 @@ pa_status pa_bm_allocate(pa_block_manager* bm, const int32_t* token_ids, int32_t
  * table back to back, ceil(length_s / block_size) entries each. *num_done: the number
  * of requests allocated. When the pool runs out at request s, the call returns
  * PA_ERR_NO_BLOCKS with *num_done = s: requests 0..s-1 keep their blocks (free them,
- * or run them), request s holds nothing. Bad offsets return PA_ERR_INVALID_ARG before
- * any block is taken. */
+ * or run them), request s holds nothing. Bad offsets and negative token ids return
+ * PA_ERR_INVALID_ARG before any block is taken. */
 pa_status pa_bm_allocate_batch(pa_block_manager* bm, const int32_t* token_ids,
                                const int32_t* cu_tokens, int32_t num_seqs,
                                const uint32_t* block_hashes, const int32_t* cu_blocks,
@@ -168,6 +170,10 @@ pa_status pa_bm_ref_counts(const pa_block_manager* bm, int32_t* out);
  *   hashes_out  uint32 [cu_blocks[num_seqs]].
  * One warp per sequence: each lane hashes whole blocks on its own, then the lanes
  * chain them with a scan (the chained hash of a prefix is a polynomial in 31).
+ * Offsets that disagree (a block count other than length_s / block_size) are
+ * clamped to the sequence's own tokens, so nothing is read past them; the hashes
+ * past the clamp are not written, and the mismatch is reported as PA_ERR_BAD_INDEX
+ * (debug checks / pa_check_device_errors).
  */
 pa_status pa_block_hashes(const int32_t* token_ids, const int32_t* cu_tokens,
                           const int32_t* cu_blocks, int32_t num_seqs, int32_t block_size,
@@ -301,9 +307,10 @@ pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* s
  * every GPU loading the library holds until the process exits. It allocates
  * nothing and calls no allocator. The caller still passes inputs and outputs.
  *
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current), which may load the
- *    library's device code; make that first call before any stream capture.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *    with the device current; a host-side lookup, so a device reset never leaves
+ *    a stale address behind). The first call on a device may load the library's
+ *    device code; make that first call before any stream capture.
  *  - Sizes whose split-K scratch (pa_decode_workspace_size for the partition
  *    used) exceeds PA_DECODE_NO_ALLOC_SCRATCH_BYTES are rejected with
  *    PA_ERR_UNSUPPORTED and nothing is launched; pass a larger partition_size

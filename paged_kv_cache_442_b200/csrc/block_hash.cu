@@ -11,6 +11,7 @@
 // and each lane rewrites its run with the prefix that precedes it. All arithmetic is
 // unsigned 32-bit, i.e. mod 2^32 like the page's mask.
 #include "pa_internal.h"
+#include "pa_ptx.cuh"
 
 namespace pa {
 namespace {
@@ -29,13 +30,24 @@ __global__ void __launch_bounds__(128) block_hash_kernel(const int32_t* __restri
                                                          const int32_t* __restrict__ cu_tokens,
                                                          const int32_t* __restrict__ cu_blocks,
                                                          int32_t num_seqs, int32_t bs,
-                                                         uint32_t* __restrict__ out) {
+                                                         uint32_t* __restrict__ out,
+                                                         unsigned* err) {
   const int s = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (s >= num_seqs) return;  // uniform per warp
   const int64_t t0 = __ldg(cu_tokens + s);
+  const int64_t ntok = static_cast<int64_t>(__ldg(cu_tokens + s + 1)) - t0;
   const int32_t first = __ldg(cu_blocks + s);
-  const int nb = __ldg(cu_blocks + s + 1) - first;
+  int nb = __ldg(cu_blocks + s + 1) - first;
+  // the block offsets must agree with the token offsets: a sequence has exactly
+  // ntok / bs full blocks. A count past that would read beyond the sequence's tokens;
+  // it is clamped (the extra output entries are left as they are) and reported.
+  const int64_t nb_max = (t0 >= 0 && ntok > 0) ? ntok / bs : 0;
+  if (nb < 0 || nb > nb_max || first < 0) {
+    if (lane == 0) flag_error(err, PA_DEV_ERR_BAD_INDEX);
+    nb = first < 0 ? 0 : static_cast<int>(nb < 0 ? 0 : nb_max);
+  }
+  if (nb == 0) return;  // uniform per warp
   uint32_t* o = out + first;
   // 1) each block's own hash (seed 0)
   for (int b = lane; b < nb; b += 32) {
@@ -79,7 +91,7 @@ cudaError_t launch_block_hashes(const int32_t* token_ids, const int32_t* cu_toke
   const int threads = 128;
   const int64_t blocks = (static_cast<int64_t>(num_seqs) * 32 + threads - 1) / threads;
   block_hash_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-      token_ids, cu_tokens, cu_blocks, num_seqs, block_size, hashes_out);
+      token_ids, cu_tokens, cu_blocks, num_seqs, block_size, hashes_out, device_error_word());
   return cudaGetLastError();
 }
 

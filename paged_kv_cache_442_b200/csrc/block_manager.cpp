@@ -216,6 +216,11 @@ pa_status pa_bm_allocate_batch(pa_block_manager* m, const int32_t* token_ids,
     if (len < 0) return PA_ERR_INVALID_ARG;
     if (len > 0 && !token_ids) return PA_ERR_INVALID_ARG;
     if (block_hashes && cu_blocks[s + 1] - cu_blocks[s] != len / bs) return PA_ERR_INVALID_ARG;
+    // token ids are checked here too, so that every PA_ERR_INVALID_ARG comes before
+    // any block is taken (pa_bm_allocate would reject a negative id only once the
+    // requests before this one hold their blocks)
+    for (int32_t i = cu_tokens[s]; i < cu_tokens[s + 1]; ++i)
+      if (token_ids[i] < 0) return PA_ERR_INVALID_ARG;
   }
   int64_t off = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {

@@ -9,11 +9,12 @@
 // GPU and held by every GPU that loads the library until the process exits.
 //
 // The array's name is only a host-side stand-in in host code, not a device address:
-// the device address is looked up with cudaGetSymbolAddress, once per device, with
-// that device current, and that address is what the kernels receive.
+// the device address is looked up with cudaGetSymbolAddress, with the device current,
+// and that address is what the kernels receive. The lookup is repeated on every call
+// (a host-side table lookup, no stream work): after a device reset the library's
+// device code is loaded again and the array may sit at another address, so a cached
+// pointer could point at memory the array no longer occupies.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -23,24 +24,12 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_decode_scratch[PA_DECODE_NO_ALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxScratchDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxScratchDevices] = {nullptr};
-
-// Device address of g_decode_scratch on the current device (looked up on first use).
+// Device address of g_decode_scratch on the current device.
 cudaError_t scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -24,7 +24,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_debug{0};
 std::mutex g_mu;
-unsigned* g_err_ptr[kMaxDevices] = {nullptr};
 int g_sm_count[kMaxDevices] = {0};
 std::set<std::pair<const void*, int>> g_smem_set;  // (kernel, device) already raised
 
@@ -64,16 +63,15 @@ pa_status finish(cudaError_t e, void* stream) {
 
 }  // namespace
 
+// Looked up on every call (a host-side table lookup): after a device reset the
+// library's device code is loaded again and the word may sit at another address.
 unsigned* device_error_word() {
-  const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_ptr[d]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_device_error_word) != cudaSuccess) return nullptr;
-    g_err_ptr[d] = static_cast<unsigned*>(ptr);
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_device_error_word) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return g_err_ptr[d];
+  return static_cast<unsigned*>(ptr);
 }
 
 int sm_count() {

@@ -196,3 +196,19 @@ def test_batch_allocation_argument_checks():
     st = lib.pa_bm_allocate_batch(bm.h, toks.ctypes.data, cu.ctypes.data, 0, None, None,
                                   out.ctypes.data, ctypes.byref(done))
     assert st == 0 and done.value == 0
+
+
+def test_batch_allocation_rejects_a_negative_token_before_taking_blocks():
+    """A negative token id in a later request fails the whole call up front: the
+    requests before it do not keep any block."""
+    import ctypes
+    bm = pa.BlockManager(16, 4)
+    lib = pa.load_library()
+    toks = np.arange(1, 11, dtype=np.int32)
+    toks[7] = -3                                   # inside the second request
+    cu = np.array([0, 6, 10], dtype=np.int32)
+    out = np.zeros(8, dtype=np.int32)
+    done = ctypes.c_int32(-1)
+    st = lib.pa_bm_allocate_batch(bm.h, toks.ctypes.data, cu.ctypes.data, 2, None, None,
+                                  out.ctypes.data, ctypes.byref(done))
+    assert st == 1 and done.value == 0 and bm.num_used() == 0

@@ -66,3 +66,30 @@ def test_gpu_hashes_give_the_same_tables():
     for s, h in zip(seqs, hs):
         assert dev.allocate(s, block_hashes=h) == host.allocate(s)
     assert np.array_equal(dev.ref_counts(), host.ref_counts())
+
+
+def test_block_offsets_past_the_tokens_are_clamped_and_reported():
+    """cu_blocks claiming one block more than a sequence's tokens hold: nothing is read
+    past the sequence (the token buffer is padded so that even an unclamped read would
+    stay inside it), the mismatch is reported, and every in-range hash is unchanged."""
+    bs = 16
+    rng = np.random.default_rng(12)
+    seqs = [rng.integers(0, 1 << 31, size=n).tolist() for n in (70, 33, 100)]
+    want = [oracle.block_hashes(s, bs) for s in seqs]
+    toks = np.concatenate([np.asarray(s, np.int32) for s in seqs] + [np.zeros(4 * bs, np.int32)])
+    lens = np.array([len(s) for s in seqs])
+    cu_t = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    nblk = lens // bs
+    nblk[1] += 1                                   # sequence 1 claims 3 blocks, has 2
+    cu_b = np.concatenate([[0], np.cumsum(nblk)]).astype(np.int32)
+    sentinel = 0x5A5A5A5A
+    out = torch.full((int(cu_b[-1]),), sentinel, dtype=torch.int32, device="cuda")
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_block_hashes(torch.from_numpy(toks).cuda(), torch.from_numpy(cu_t).cuda(),
+                           torch.from_numpy(cu_b).cuda(), bs, out)
+    assert e.value.status == 3
+    h = out.cpu().numpy().view(np.uint32)
+    assert np.array_equal(h[cu_b[0]:cu_b[1]], want[0])
+    assert np.array_equal(h[cu_b[1]:cu_b[1] + 2], want[1])
+    assert h[cu_b[1] + 2] == sentinel               # the claimed third block is not written
+    assert np.array_equal(h[cu_b[2]:cu_b[3]], want[2])

@@ -4,7 +4,7 @@ import pytest
 
 from tests.gpu_helpers import (DeviceWorkload, assert_close, oracle_decode, oracle_pools,
                                oracle_prefill, to_bits, to_f64)
-from workloads import CONFIGS, build_workload, generate
+from workloads import CONFIGS, build_workload, generate, relabel_blocks
 
 import oracle
 
@@ -71,3 +71,17 @@ def test_prefill_is_deterministic():
     w = generate(CONFIGS["chunked_prefill"], num_seqs=4)
     dw = DeviceWorkload(w)
     assert np.array_equal(to_bits(dw.prefill()), to_bits(dw.prefill()))
+
+
+@pytest.mark.parametrize("bs", [64, 256])
+def test_prefill_block_permutation_is_bitwise_invariant(bs):
+    """Relabelling the physical blocks (data and tables moved together) gives the same
+    bits: the kernel's arithmetic depends only on logical positions."""
+    ctx = np.array([700, 300, 1000, 129])
+    new = np.array([200, 300, 129, 1])
+    w = build_workload(kind="prefill", context_lens=ctx, new_lens=new, num_q_heads=8,
+                       num_kv_heads=2, head_dim=128, block_size=bs, seed=900 + bs)
+    perm = np.random.default_rng(bs).permutation(w.num_blocks)
+    a = to_bits(DeviceWorkload(w).prefill())
+    b = to_bits(DeviceWorkload(relabel_blocks(w, perm)).prefill())
+    assert np.array_equal(a, b)

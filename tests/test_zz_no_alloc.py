@@ -3,9 +3,10 @@
 Such callers (a runtime that fixes all of its GPU memory at start-up, or a host
 program that only binds the C ABI and has no CUDA allocator) cannot hand pa_decode
 a workspace; this entry point uses the library's own fixed scratch array instead.
-The test drives it through the C ABI and checks it against pa_decode (which gets
-a caller-allocated workspace) on two calls in a row with different workloads, so
-the second call runs on whatever the first left in the shared array.
+The test drives it through the C ABI and checks it on two calls in a row with
+different workloads, so the second call runs on whatever the first left in the
+shared array: bit for bit against pa_decode (which gets a caller-allocated
+workspace) at the same partition size, and against the oracle within the bar.
 
 Kept in its own file, named to be collected after every other test.
 """
@@ -14,7 +15,7 @@ import pytest
 import torch
 
 import paged_kv_cache_442_b200 as pa
-from tests.gpu_helpers import DeviceWorkload, assert_close, to_f64
+from tests.gpu_helpers import DeviceWorkload, assert_close, oracle_decode, to_bits
 from workloads import CONFIGS, generate
 
 pytestmark = pytest.mark.gpu
@@ -29,6 +30,9 @@ def _no_alloc(dw):
 
 
 def test_no_alloc_decode_matches_workspace_decode_on_two_calls():
+    """Two calls in a row (the second runs on whatever the first left in the shared
+    array): each equals pa_decode at the same partition size bit for bit, and matches
+    the oracle within the decode bar."""
     first = DeviceWorkload(generate(CONFIGS["decode_b64"]))
     second = DeviceWorkload(generate(CONFIGS["long_ctx_decode"]))
     for dw in (first, second):
@@ -37,12 +41,19 @@ def test_no_alloc_decode_matches_workspace_decode_on_two_calls():
         need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim,
                                            w.max_context_len, P)
         assert 0 < need <= pa.DECODE_NO_ALLOC_SCRATCH_BYTES  # both calls really use the scratch
-    ref1, ref2 = to_f64(first.decode()), to_f64(second.decode())
-    got1 = to_f64(_no_alloc(first))
-    got2 = to_f64(_no_alloc(second))
+        assert P < w.max_context_len                         # and both split their contexts
+    ref1, ref2 = to_bits(first.decode()), to_bits(second.decode())
+    got1 = to_bits(_no_alloc(first))
+    got2 = to_bits(_no_alloc(second))
     torch.cuda.synchronize()
-    assert_close(got1, ref1, "no-alloc call 1 vs pa_decode")
-    assert_close(got2, ref2, "no-alloc call 2 vs pa_decode")
+    assert np.array_equal(got1, ref1), "no-alloc call 1 differs from pa_decode"
+    assert np.array_equal(got2, ref2), "no-alloc call 2 differs from pa_decode"
+    assert_close(bits_to_f64(got1), oracle_decode(first.w), "no-alloc call 1 vs oracle")
+    assert_close(bits_to_f64(got2), oracle_decode(second.w), "no-alloc call 2 vs oracle")
+
+
+def bits_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def test_no_alloc_rejects_sizes_beyond_its_scratch():
