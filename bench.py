@@ -166,8 +166,10 @@ def prefill_bytes(w):
 
 # --------------------------------------------------------------------------- GPU arm
 class GpuRunner:
-    def __init__(self, w, torch, pa, partition_size=0, separate_store=False, cow=None):
+    def __init__(self, w, torch, pa, partition_size=0, separate_store=False, cow=None,
+                 shared_len=0):
         self.w, self.torch, self.pa = w, torch, pa
+        self.shared_len = shared_len
         dev = torch.device("cuda")
         shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         fill = int(np.uint16(SENTINEL_BF16).view(np.int16))
@@ -196,7 +198,15 @@ class GpuRunner:
         self.context_lens = i32(w.context_lens)
         self.cu = i32(w.cu_seqlens_q)
         self.out = torch.empty_like(self.q)
-        if w.kind == "decode":
+        if w.kind == "decode" and shared_len:
+            # the shared prefix attended once (its blocks: the longest sequence's first
+            # ones, held by every sequence), then the rest of every context
+            s_long = int(np.argmax(w.context_lens))
+            self.shared_blocks = i32(w.block_tables[s_long, :shared_len // w.block_size])
+            self.ws, self.P = pa.shared_prefix_workspace(
+                w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.max_context_len,
+                shared_len, partition_size)
+        elif w.kind == "decode":
             self.ws, self.P = pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads,
                                                   w.head_dim, w.max_context_len, partition_size)
             # kernels one pa_decode launches: the persistent tcgen05 kernel merges its
@@ -207,12 +217,15 @@ class GpuRunner:
                   and self.P <= 2048)
             split = self.P < w.max_context_len
             self.decode_launches = 1 if tc or not split else 2
-        # a decode step that stores new tokens runs as one pa_store_decode call (the
-        # tensor-core kernel stores the rows itself; other shapes add a store launch)
-        self.fused = w.kind == "decode" and self.new_k is not None and not separate_store
+            if shared_len:
+                self.decode_launches = 2 if w.max_context_len > shared_len else 1
+        # a step that stores new tokens runs as one pa_store_decode / pa_store_prefill
+        # call (the kernel stores the rows itself; decode shapes off the tensor-core
+        # path add a store launch)
+        self.fused = self.new_k is not None and not separate_store
         # copy-on-write pairs copied before each step (blocks the step appends into)
         self.cow = None if cow is None else (i32(cow[0]), i32(cow[1]))
-        if self.fused and not tc:
+        if self.fused and w.kind == "decode" and not tc:
             self.decode_launches += 1
         self.max_q = int(np.max(np.diff(w.cu_seqlens_q))) if w.num_seqs else 0
         torch.cuda.synchronize()
@@ -234,10 +247,20 @@ class GpuRunner:
         out = self.out if out is None else out
         ctx = self.context_lens if ctx is None else ctx
         bt = self.block_tables if bt is None else bt
-        if self.fused:
+        if self.fused and w.kind == "decode":
             pa.pa_store_decode(self.new_k if k is None else k, self.new_v if v is None else v,
                                self.new_slots if slots is None else slots, out, q, self.k_cache,
                                self.v_cache, bt, ctx, w.scale, w.max_context_len, self.P, self.ws)
+            return self.decode_launches
+        if self.fused:
+            pa.pa_store_prefill(self.new_k if k is None else k, self.new_v if v is None else v,
+                                self.new_slots if slots is None else slots, out, q, self.k_cache,
+                                self.v_cache, bt, self.cu, ctx, w.scale, self.max_q)
+            return 1
+        if w.kind == "decode" and self.shared_len:
+            pa.pa_decode_shared_prefix(out, q, self.k_cache, self.v_cache, bt, ctx, w.scale,
+                                       w.max_context_len, self.shared_blocks, self.shared_len,
+                                       self.P, self.ws)
             return self.decode_launches
         if w.kind == "decode":
             pa.pa_decode(out, q, self.k_cache, self.v_cache, bt, ctx, w.scale,
@@ -827,7 +850,9 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
             cow = (src, dst)
         else:
             w = generate(CONFIGS[name])
-        r = GpuRunner(w, torch, pa, cow=cow)
+        # prefill: the attention kernel alone after a separate store (its roofline),
+        # then the step as one pa_store_prefill launch
+        r = GpuRunner(w, torch, pa, cow=cow, separate_store=(w.kind == "prefill"))
         n = steps if w.kind == "decode" else 50
         total_ms, attn_ms, lps = time_steps(r, torch, n, warmup, flush)
         a_ms = sum(attn_ms) / len(attn_ms)
@@ -853,6 +878,23 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
                 ub = w.kv_bytes_unique() + 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
                 d.update({"unique_bytes": ub, "unique_GBps": round(ub / a_ms / 1e6, 1),
                           "frac_of_hbm_peak_unique": round(ub / a_ms / 1e6 / hbm_peak, 3)})
+            if name == "prefix_share_decode":
+                # the same batch with its shared prefix attended once for all sequences
+                del r
+                torch.cuda.empty_cache()
+                S = CONFIGS[name].shared_prefix_len
+                r = GpuRunner(w, torch, pa, shared_len=S)
+                s_ms, s_attn, s_lps = time_steps(r, torch, n, warmup, flush)
+                sa = sum(s_attn) / len(s_attn)
+                d["shared_prefix"] = {
+                    "kernel": "pa_decode_shared_prefix (dense tcgen05 pass over the shared "
+                              "prefix + persistent decode of the rest)",
+                    "shared_len": S, "attn_us": round(sa * 1e3, 2), "launches": s_lps,
+                    "partition_size": r.P,
+                    "logical_GBps": round(lb / sa / 1e6, 1),
+                    "unique_GBps": round(ub / sa / 1e6, 1),
+                    "frac_of_hbm_peak_unique": round(ub / sa / 1e6 / hbm_peak, 3),
+                    "speedup_vs_pa_decode": round(a_ms / sa, 3)}
         else:
             fl = prefill_flops(w)
             st_ms = total_ms / n - a_ms
@@ -861,7 +903,17 @@ def measure_others(torch, pa, hbm_peak, tf_peak, tf_sustained, peak_src, steps=2
                       "frac_of_bf16_peak_sustained": round(fl / a_ms / 1e9 / tf_sustained, 3),
                       "frac_of_bf16_peak_burst": round(fl / a_ms / 1e9 / tf_peak, 3),
                       "store_us": round(st_ms * 1e3, 2),
-                      "store_GBps": round(store_bytes(w) / st_ms / 1e6, 1)})
+                      "store_GBps": round(store_bytes(w) / st_ms / 1e6, 1),
+                      "separate_store_step_us": round(total_ms / n * 1e3, 2)})
+            del r
+            torch.cuda.empty_cache()
+            r = GpuRunner(w, torch, pa)
+            f_ms, f_attn, f_lps = time_steps(r, torch, n, warmup, flush)
+            fa = sum(f_attn) / len(f_attn)
+            d.update({"step_us": round(f_ms / n * 1e3, 2), "step_launches": f_lps,
+                      "step": "one pa_store_prefill launch (new rows stored by the attention "
+                              "kernel)",
+                      "step_TFLOPs": round(fl / fa / 1e9, 1)})
         d["peak_source"] = peak_src
         res[name] = d
         del r

@@ -294,6 +294,43 @@ pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* s
                           size_t workspace_bytes, void* stream);
 
 /*
+ * pa_decode_shared_prefix — pa_decode for a batch whose sequences all start with the
+ * same shared_len positions held in the same physical blocks (nano vllm page, section
+ * 3.2.2: requests with a common prompt share reference-counted blocks; the block
+ * manager that handed them out knows how long the common part is). The shared
+ * prefix is attended once for all sequences: one dense tensor-core pass per kv head
+ * over every sequence's query rows (each row sees min(context_lens[s], shared_len)
+ * of the prefix), whose result is the output row of a context that ends inside the
+ * prefix and the first split-K partial of a longer one; the persistent decode then
+ * reads only the positions past the prefix and merges. Two launches on `stream`.
+ *
+ *   shared_blocks  int32 [shared_len / block_size], device: the physical blocks of
+ *                  the shared prefix. Every sequence's block table must hold them at
+ *                  the prefix positions it uses (b * block_size < context_lens[s]); a
+ *                  difference is reported as PA_ERR_BAD_INDEX. The prefix is read
+ *                  through shared_blocks.
+ *   shared_len     a multiple of 128 (0 = pa_decode).
+ *   workspace      at least pa_decode_shared_prefix_workspace_size(...) bytes for the
+ *                  partition size used (partition_size 0 = automatic, sized on the
+ *                  positions past the prefix).
+ *   other arguments as pa_decode. Supported: head_dim 128, Hq / Hkv in {1, 2, 4, 8,
+ *   16}, partition_size a multiple of 128 up to 2048; else PA_ERR_UNSUPPORTED.
+ * The result equals pa_decode's within the same rounding (the positions are summed in
+ * another grouping); CUDA graphs: as pa_decode (clear the counter block).
+ */
+size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t head_dim, int32_t max_context_len,
+                                              int32_t shared_len, int32_t partition_size);
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, pa_cache_desc cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, float scale, int32_t max_context_len,
+                                  const int32_t* shared_blocks, int32_t shared_len,
+                                  int32_t partition_size, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * pa_decode_no_alloc — pa_decode for callers that cannot allocate device memory.
  * (The pages have no counterpart: this is an interface convenience, not a step of
  * the method.)
@@ -359,11 +396,15 @@ pa_status pa_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void
 
 /*
  * pa_decode_fp8 — pa_decode over e4m3 pools: the attention of the values the
- * pools hold (code * scale). Each K/V tile is loaded as codes and scales,
- * dequantised to bf16 (code * scale rounded once to nearest even) in shared memory,
- * and then takes pa_decode's tensor-core path unchanged. Arguments as pa_decode,
- * with the pools replaced by codes and scales (16-byte aligned).
- * Supported: head_dim 128, Hq / Hkv in {1, 2, 4, 8}, partition_size (given or
+ * pools hold (code * scale). The tensor cores read the stored codes directly
+ * (e4m3 x e4m3 products, fp32 accumulation); no code is converted. Each row's K
+ * scale multiplies that position's score, and each row's V scale its probability,
+ * in fp32. q and the probabilities reach the tensor cores as two e4m3 terms each
+ * (a high term and the rounded remainder), which keeps about 2^-8 relative
+ * accuracy per element. Arguments as pa_decode, with the pools replaced by codes
+ * and scales (16-byte aligned). Values whose products overflow fp32 are out of
+ * range (as for pa_decode).
+ * Supported: head_dim 128, Hq / Hkv in {1, 2, 4, 8, 16}, partition_size (given or
  * automatic) a multiple of 128 up to 2048; anything else returns
  * PA_ERR_UNSUPPORTED (there is no CUDA-core fp8 path).
  */
@@ -399,10 +440,51 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
                      int32_t total_q, int32_t max_q_len, float scale, void* stream);
 
 /*
+ * pa_store_prefill — one chunked-prefill step of a layer in one call: store the new
+ * tokens' K/V rows, then attend (nano vllm page, section 3.1: the new tokens follow
+ * the num_cached_tokens of a Sequence in its blocks; mini-vllm page, section 2: K/V are
+ * written where the block table points, then read through it). The result, and the
+ * pool afterwards, equal pa_store_kvcache followed by pa_prefill with the same
+ * arguments.
+ *
+ *   new_k, new_v   [total_q, Hkv, D] bf16: the K and V rows of the new tokens, in the
+ *                  token order of q (sequence s owns rows cu_seqlens_q[s] ..).
+ *   slot_mapping   int32 [total_q]: the slot of each new token, which must be the slot
+ *                  the block table gives for its position (context_lens[s] - n_new + i
+ *                  for new token i of sequence s), or -1 (not stored). Any other value
+ *                  is not stored and is reported as PA_ERR_BAD_INDEX (debug checks /
+ *                  pa_check_device_errors).
+ *   other arguments as pa_prefill.
+ * The attention reads the new tokens' rows from new_k / new_v directly (the bits the
+ * store writes), so the launch has no ordering between its store and its reads; the
+ * rows reach the pool in the same launch. A slot of -1 therefore still attends to the
+ * row in new_k / new_v (store then prefill would read the pool's old row there).
+ */
+pa_status pa_store_prefill(const void* new_k, const void* new_v, const int32_t* slot_mapping,
+                           void* out, const void* q, void* k_cache, void* v_cache,
+                           pa_cache_desc cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* cu_seqlens_q,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t total_q, int32_t max_q_len, float scale, void* stream);
+
+/*
  * Debug mode: when on, every entry point synchronises its stream after the
  * launch and returns the device error status (see pa_check_device_errors).
  */
 void pa_set_debug_checks(int on);
+
+/*
+ * Test hook: the time limit, in nanoseconds, of the waits between the cooperating
+ * roles (data movement, tensor-core issue, softmax, epilogue) inside the
+ * tensor-core kernels of later calls; 0 restores the default of 2 s. A wait that
+ * runs out records PA_ERR_TIMEOUT in the device error word and the kernel winds
+ * down: every role leaves its loop, each CTA still waits (with the full 2 s limit)
+ * for the copies and tensor-core operations it has started, frees its tensor
+ * memory and returns, so the context stays usable and the next call is a normal
+ * one. Outputs of a call that timed out are unspecified. Exists so that tests can
+ * make a wait run out without a fault; a serving process leaves it alone.
+ */
+void pa_set_wait_limit_ns(uint64_t ns);
 
 /*
  * Synchronise `stream`, read and clear this device's error word.

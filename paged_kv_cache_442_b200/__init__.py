@@ -23,8 +23,9 @@ EXPORTED = ("pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_allocate_b
             "pa_bm_append",
             "pa_bm_num_used", "pa_bm_ref_counts", "pa_block_hashes",
             "pa_store_kvcache", "pa_copy_blocks", "pa_decode_default_partition", "pa_decode_workspace_size",
-            "pa_decode", "pa_store_decode", "pa_decode_no_alloc", "pa_prefill",
-            "pa_store_kvcache_fp8", "pa_decode_fp8", "pa_set_debug_checks",
+            "pa_decode", "pa_store_decode", "pa_decode_shared_prefix",
+            "pa_decode_shared_prefix_workspace_size", "pa_decode_no_alloc", "pa_prefill", "pa_store_prefill",
+            "pa_store_kvcache_fp8", "pa_decode_fp8", "pa_set_debug_checks", "pa_set_wait_limit_ns",
             "pa_check_device_errors", "pa_status_string", "pa_version")
 
 # size of the library-owned scratch of pa_decode_no_alloc (include/pa.h)
@@ -89,12 +90,20 @@ def load_library(path: str | None = None):
     lib.pa_store_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
                                     ctypes.c_float, i32, i32, vp, sz, vp]
     lib.pa_store_decode.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
+                                            ctypes.c_float, i32, vp, i32, i32, vp, sz, vp]
+    lib.pa_decode_shared_prefix.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.pa_decode_shared_prefix_workspace_size.restype = sz
     lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
                                        ctypes.c_float, i32, i32, vp]
     lib.pa_decode_no_alloc.restype = ctypes.c_int
     lib.pa_prefill.argtypes = [vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, vp, i32, i32, i32, i32,
                                ctypes.c_float, vp]
     lib.pa_prefill.restype = ctypes.c_int
+    lib.pa_store_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, vp, i32,
+                                     i32, i32, i32, ctypes.c_float, vp]
+    lib.pa_store_prefill.restype = ctypes.c_int
     lib.pa_store_kvcache_fp8.argtypes = [vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp]
     lib.pa_store_kvcache_fp8.restype = ctypes.c_int
     lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, pa_cache_desc, vp, i32, vp, i32, i32,
@@ -102,6 +111,8 @@ def load_library(path: str | None = None):
     lib.pa_decode_fp8.restype = ctypes.c_int
     lib.pa_set_debug_checks.argtypes = [ctypes.c_int]
     lib.pa_set_debug_checks.restype = None
+    lib.pa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.pa_set_wait_limit_ns.restype = None
     lib.pa_check_device_errors.argtypes = [vp]
     lib.pa_check_device_errors.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -438,6 +449,53 @@ def pa_store_decode(new_k, new_v, slot_mapping, out, q, k_cache, v_cache, block_
     _raise("pa_store_decode", st)
 
 
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                            max_context_len: int, shared_blocks, shared_len: int,
+                            partition_size: int = 0, workspace=None, stream=None) -> None:
+    """Decode of a batch whose first shared_len positions live in the same blocks
+    (shared_blocks, int32 device tensor) for every sequence: the shared prefix attended
+    once for all of them, then the rest."""
+    torch = _torch()
+    lib = load_library()
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    _check(shared_blocks, "shared_blocks", torch.int32, 1)
+    B, Hq, D = q.shape
+    if tuple(out.shape) != (B, Hq, D) or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("out/q/block_tables/context_lens disagree on num_seqs")
+    if shared_len and shared_blocks.shape[0] * k_cache.shape[1] < shared_len:
+        raise ValueError("shared_blocks must cover shared_len positions")
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_shared_prefix(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     cache_desc(k_cache), _ptr(block_tables),
+                                     int(block_tables.shape[1]), _ptr(context_lens), int(B), int(Hq),
+                                     float(scale), int(max_context_len), _ptr(shared_blocks),
+                                     int(shared_len), int(partition_size),
+                                     _ptr(workspace) if workspace is not None else ctypes.c_void_p(0),
+                                     ws_bytes, _stream(stream))
+    _raise("pa_decode_shared_prefix", st)
+
+
+def shared_prefix_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                            shared_len, partition_size=0, device="cuda"):
+    """Allocate (with torch) the scratch pa_decode_shared_prefix needs; returns
+    (workspace, partition size) as decode_workspace does."""
+    torch = _torch()
+    lib = load_library()
+    rest = max(1, max_context_len - shared_len)
+    P = partition_size or pa_decode_default_partition(num_seqs, num_kv_heads, rest)
+    nbytes = int(lib.pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim,
+                                                            max_context_len, shared_len, P))
+    return torch.empty(max(nbytes, 16) // 4, dtype=torch.float32, device=device), P
+
+
 def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
                        max_context_len: int, partition_size: int = 0, stream=None) -> None:
     """pa_decode for callers that cannot allocate device memory.
@@ -495,8 +553,46 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, cu_seqlens_q, context_len
     _raise("pa_prefill", st)
 
 
+def pa_store_prefill(new_k, new_v, slot_mapping, out, q, k_cache, v_cache, block_tables,
+                     cu_seqlens_q, context_lens, scale: float, max_q_len: int,
+                     stream=None) -> None:
+    """Store the new tokens' K/V rows at slot_mapping (their block-table slots) and run
+    the causal paged prefill in one launch: the same result, and pool, as
+    pa_store_kvcache followed by pa_prefill."""
+    torch = _torch()
+    lib = load_library()
+    _check(new_k, "new_k", torch.bfloat16, 3)
+    _check(new_v, "new_v", torch.bfloat16, 3)
+    _check(slot_mapping, "slot_mapping", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _check(context_lens, "context_lens", torch.int32, 1)
+    Tq, Hq, D = q.shape
+    B = context_lens.shape[0]
+    if tuple(out.shape) != (Tq, Hq, D) or cu_seqlens_q.shape[0] != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("out/q/cu_seqlens_q/block_tables/context_lens shapes disagree")
+    row = (Tq, k_cache.shape[2], k_cache.shape[3])
+    if tuple(new_k.shape) != row or tuple(new_v.shape) != row or slot_mapping.shape[0] != Tq:
+        raise ValueError("new_k/new_v must be [total_q, Hkv, D] and slot_mapping [total_q]")
+    st = lib.pa_store_prefill(_ptr(new_k), _ptr(new_v), _ptr(slot_mapping), _ptr(out), _ptr(q),
+                              _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
+                              int(block_tables.shape[1]), _ptr(cu_seqlens_q), _ptr(context_lens),
+                              int(B), int(Hq), int(Tq), int(max_q_len), float(scale), _stream(stream))
+    _raise("pa_store_prefill", st)
+
+
 def pa_set_debug_checks(on: bool) -> None:
     load_library().pa_set_debug_checks(1 if on else 0)
+
+
+def pa_set_wait_limit_ns(ns: int) -> None:
+    """Test hook: bound of the waits between the tensor-core kernels' roles (0 = the
+    default 2 s). See include/pa.h."""
+    load_library().pa_set_wait_limit_ns(int(ns))
 
 
 def pa_check_device_errors(stream=None) -> int:

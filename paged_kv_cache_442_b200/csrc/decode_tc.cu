@@ -16,18 +16,17 @@
 //           item ahead of the producer;
 //   warp 4  producer: loads q (one box per item) and the K and V tiles
 //           of 128 positions through the block table (one TMA box per physical
-//           block) into two 3-deep rings of 32 KB slots. A K slot frees as soon as
-//           its score MMA is done and a V slot when its value MMA is done, so both
-//           streams run about two tiles ahead of the consumers (the fetch latency,
-//           ~1.4 us per tile, must overlap; a shared K+V slot held until the value MMA
-//           left one tile in flight);
+//           block) into a K ring and a V ring. A K slot frees as soon as its score
+//           MMA is done and a V slot when its value MMA is done, so both streams run
+//           several tiles ahead of the consumers (the fetch latency, ~1.4 us per tile,
+//           must overlap);
 //   warp 5  tensor-core issuer: owns the TMEM allocation; for tile j it issues S^T(j)
 //           and then O^T += V^T P^T for tile j-1, and the last tile's value MMA of an
 //           item right away so the item's epilogue never waits on the next item;
 //   warps 0-3  softmax: thread r owns position r of a tile (TMEM lane r): per-head
 //           tile max across the 128 positions, exp2 against a per-item reference max,
-//           P^T to shared memory as bf16. O^T is rescaled in TMEM only when a tile's
-//           max exceeds the reference by more than 2^8 (so probabilities stay <= 256,
+//           P^T to shared memory. O^T is rescaled in TMEM only when a tile's max
+//           exceeds the reference by more than 2^8 (so probabilities stay <= 256,
 //           exact in fp32 and bf16 range) — the only step that waits for the previous
 //           value MMA. At the end of an item they post (m, l) and move on;
 //   warps 6-9  epilogue: thread d owns output dim d (TMEM lane d) of the item's O^T
@@ -38,21 +37,30 @@
 // Counters in the workspace carry a per-call tag, so an earlier call's leftovers never
 // count: the workspace needs no clearing between calls.
 //
-// fp8 variant (pa_decode_fp8): the pools hold e4m3 codes with one fp32 scale per
-// (position, kv head) row. The producer loads a tile's codes into the upper half of
-// its 32 KB ring slot and the tile's scales (one box per block, each on a 128-byte
-// boundary) into a small area of the slot's own; converter warps (11-18 for up to 4
-// query heads per kv head, two threads per row; 11-14 for 8, one thread per row)
-// dequantise it in place: one of them waits for the bytes while the rest sleep in a
-// named barrier, each thread reads its share of a row's 128 codes and the row's scale
-// into registers, and after a warp sync (a row's upper-half bf16 covers only its own
-// codes) writes the row as bf16 (code * scale, rounded once) into both swizzled
-// halves. The score, softmax, value and merge stages are the bf16 ones, unchanged.
+// e4m3 pools (pa_decode_fp8): the tensor cores read the codes as they are stored
+// (tcgen05.mma kind::f8f6f4: K tiles K-major, V tiles as the MN-major A operand of
+// the value product, both 128-byte-swizzled by TMA), so no code is ever converted.
+// Each row's scale is applied where its index is a free dimension of the product:
+//   * a K row scale multiplies that position's score column in the softmax;
+//   * a V row scale multiplies that position's probability before P^T is written:
+//     P'_j = 2^(x_j + log2 s_v,j - R), with R a per-item, per-head reference kept so
+//     that P' <= 2^6 (O^T is rescaled when a tile would exceed that, as for the max);
+//     l keeps summing 2^(x_j - m) in fp32, and the output is O^T 2^(R - m) / l;
+//   * q (bf16) becomes two e4m3 terms with one fp32 scale per head, hi = e4m3(q/s)
+//     and lo = e4m3(q/s - hi), written by the scheduler warp; S^T accumulates
+//     K hi^T + K lo^T (about 2^-8 relative error on each q element);
+//   * P' becomes hi = e4m3(P') and lo = e4m3(128 (P' - hi)), accumulated into two
+//     O^T accumulators combined as O_hi + O_lo / 128 (about 2^-8 relative on P', and
+//     an absolute floor near 2^-17, so small probabilities keep their precision).
+// Before a CTA ends, its producer waits for every copy it started and its issuer for
+// every MMA it issued (with the full time limit, even when the roles gave up early),
+// so no asynchronous write outlives the CTA's shared and tensor memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include <atomic>
+#include <cfloat>
 #include <ctime>
 
 #include "pa_internal.h"
@@ -64,8 +72,6 @@ namespace {
 constexpr int TM = 128;        // positions per tile
 constexpr int HD = 128;        // head dim
 constexpr int NQ = 16;         // MMA N: query heads of one kv head, padded
-constexpr int NK = 3;          // K ring depth (a slot frees when its score MMA is done)
-constexpr int NV = 3;          // V ring depth (a slot frees when its value MMA is done)
 constexpr int NS = 4;          // S^T buffers in TMEM
 constexpr int NP = 4;          // P^T buffers in shared memory
 constexpr int QN = 2;          // item queue depth (producer -> issuer, softmax)
@@ -73,64 +79,73 @@ constexpr int QS = 2;          // scheduler queue depth: one item prepared ahead
                                // queues reserve work early and unbalance the tail)
 constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flight)
 constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
-constexpr int kConvWarp0 = 11;   // fp8 pools: converter warps follow the scheduler
-// fp8: 8 converter warps (two threads per row of a tile) where the other roles fit in
-// the registers that leaves (608 threads: up to 4 query heads per kv head), else 4
-template <int G>
-constexpr int conv_warps() { return G <= 4 ? 8 : 4; }
-template <int G, bool F8>
-constexpr int tc_threads() { return kThreads + (F8 ? 32 * conv_warps<G>() : 0); }
-constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more than this
-constexpr int kRegion = TM * 128;            // 64 head dims x 128 positions (16 KB)
-constexpr int kTileBytes = 2 * kRegion;      // one K or V tile (32 KB)
-constexpr int kQRegion = NQ * 128;           // 16 rows x 64 elements (2 KB)
-constexpr int kQBytes = 2 * kQRegion;
-constexpr int kPBytes = 2 * kQRegion;        // P^T: 16 heads x 128 positions, bf16
+constexpr float kRescaleLog2 = 8.f;  // rescale when the max grows by more than this
+constexpr int kQRegion = NQ * 128;           // 16 rows x 128 bytes (2 KB)
+constexpr int kQBytes = 2 * kQRegion;        // bf16: two 64-dim halves; e4m3: hi, lo terms
+constexpr int kPBytes = 2 * kQRegion;        // bf16: P^T 16 x 128; e4m3: hi, lo terms
 constexpr int kMaxIds = 2048 / 16 + 2;       // block ids of one item (partition <= 2048)
+constexpr int kSclBytes = 1024;              // e4m3: one tile's row scales (<= 8 boxes)
+constexpr int kEpiBytes = 32 + 3 * NQ * 4;   // descriptor, m, l, e4m3 output factor
+// e4m3 value path: P' <= 2^kPBoundLog2 (a rescale brings the bound to 2^kPTargetLog2),
+// so its low term, scaled by kPLoScale, stays inside e4m3's range (|128 (P' - hi)| <=
+// 128 * 2 = 256 < 448)
+constexpr float kPBoundLog2 = 6.f;
+constexpr float kPTargetLog2 = 1.f;
+constexpr float kPLoScale = 128.f;
 
 constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// every region starts on a 16-byte boundary (1024 for the swizzled operand tiles);
-// the static_asserts below keep it that way when depths change
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + NK * kTileBytes;
-constexpr int kOffQ = kOffV + NV * kTileBytes;
-constexpr int kOffP = kOffQ + QN * kQBytes;
-constexpr int kOffRed = kOffP + NP * kPBytes;                     // [3][4 warps][NQ] floats
-constexpr int kOffIds = align_up(kOffRed + 3 * 4 * NQ * 4, 16);
-constexpr int kOffSched = align_up(kOffIds + QS * kMaxIds * 4, 16);  // [QS] descriptors
-constexpr int kOffSchedFb = align_up(kOffSched + QS * 32, 16);       // [QS] first blocks
-constexpr int kOffDesc = align_up(kOffSchedFb + QS * 4, 16);         // [QN] item descriptors
-constexpr int kOffEpi = align_up(kOffDesc + QN * 32, 16);            // [NO] hand-offs
-constexpr int kEpiBytes = 32 + 2 * NQ * 4;                           // descriptor, m, l
-constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
-constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS + NK + NV;
-constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;
-// fp8 only: each K / V ring slot's row scales are staged in a 1 KB area of their own
-// (one 128-byte-aligned box per block; block size >= 16 gives at most 8 boxes), so
-// converting a slot in place never overwrites scales another thread still has to read
-constexpr int kSclBytes = 1024;
-constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
-constexpr int kSmemBytesF8 = kOffScl + (NK + NV) * kSclBytes + 1024;
-static_assert(kSmemBytesF8 <= 227 * 1024, "shared memory per CTA (fp8)");
-static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
-              "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
-static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "tile sizes");
-static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
-static_assert(kOffSched % 16 == 0 && kOffDesc % 16 == 0 && kOffEpi % 16 == 0 && kEpiBytes % 16 == 0,
-              "descriptor slots");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+// Shared-memory layout and ring depths of the bf16 (F8 = false) and e4m3 kernels.
+// Every region starts on a 16-byte boundary (1024 for the swizzled operand tiles);
+// the static_asserts below keep it that way when depths change.
+template <bool F8>
+struct Cfg {
+  static constexpr int kRegion = TM * 128;                    // 128 rows x 128 bytes
+  static constexpr int kTileBytes = F8 ? kRegion : 2 * kRegion;  // one K or V tile
+  static constexpr int NK = F8 ? 5 : 3;  // K ring (a slot frees when its score MMA is done)
+  static constexpr int NV = F8 ? 6 : 3;  // V ring (a slot frees when its value MMA is done)
+  static constexpr int NSC = F8 ? 8 : 1;  // e4m3: K-scale ring (freed by the softmax); unused for bf16
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + NK * kTileBytes;
+  static constexpr int kOffQ = kOffV + NV * kTileBytes;
+  static constexpr int kOffP = kOffQ + QN * kQBytes;
+  static constexpr int kOffRed = kOffP + NP * kPBytes;  // [3][4 warps][NQ] + [2][4] floats
+  static constexpr int kRedFloats = 3 * 4 * NQ + 2 * 4;
+  static constexpr int kOffQs = align_up(kOffRed + kRedFloats * 4, 16);  // [QN][NQ] q scales
+  static constexpr int kOffIds = align_up(kOffQs + QN * NQ * 4, 16);
+  static constexpr int kOffSched = align_up(kOffIds + QS * kMaxIds * 4, 16);  // [QS] descriptors
+  static constexpr int kOffSchedFb = align_up(kOffSched + QS * 32, 16);       // [QS] first blocks
+  static constexpr int kOffDesc = align_up(kOffSchedFb + QS * 4, 16);         // [QN] item descriptors
+  static constexpr int kOffEpi = align_up(kOffDesc + QN * 32, 16);            // [NO] hand-offs
+  static constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
+  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS +
+                                  1 + (F8 ? 2 * NSC + NV : 0);
+  static constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
+  // e4m3: the K-scale ring [NSC] and each V slot's scales [NV], 1 KB each
+  static constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
+  static constexpr int kSmemBytes = (F8 ? kOffScl + (NSC + NV) * kSclBytes : kOffMisc + 64) + 1024;
+  // TMEM columns: S^T[NS] at 16 i; O^T[NO] at 64 + 16 i; e4m3 low-term O^T at 112 + 16 i
+  static constexpr uint32_t kTmemO = 64;
+  static constexpr uint32_t kTmemOlo = 64 + 16 * NO;
+  static constexpr uint32_t kTmemCols = F8 ? 256 : 128;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
+                "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
+  static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "tile sizes");
+  static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(kOffSched % 16 == 0 && kOffDesc % 16 == 0 && kOffEpi % 16 == 0 && kEpiBytes % 16 == 0,
+                "descriptor slots");
+  static_assert(kTmemOlo + (F8 ? 16 * NO : 0) <= kTmemCols && kTmemO + 16 * NO <= kTmemCols,
+                "tensor memory columns");
+};
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kTmemCols = 128;  // S[NS] at 16*i; O[NO] at 64 + 16*i
-constexpr uint32_t kTmemO = 64;
-static_assert(kTmemO + 16 * NO <= kTmemCols, "tensor memory columns");
 
 constexpr unsigned kCountBits = 24;
 constexpr unsigned long long kCountMask = (1ull << kCountBits) - 1;
 
 struct TcParams {
   __nv_bfloat16* out;
+  const __nv_bfloat16* q;        // [B, Hq, D] (read by the scheduler for e4m3 pools)
   const int32_t* block_tables;
   const int32_t* context_lens;
   unsigned long long* counters;  // [0]: work counter, [1 + s*Hq + g*G]: arrivals of (s, g)
@@ -138,6 +153,7 @@ struct TcParams {
   float* ws_ml;                  // [B, Hq, max_parts, 2]
   unsigned* err;
   unsigned long long tag;        // per-call epoch (< 2^40, never 0)
+  unsigned long long wait_ns;    // bound of the waits between roles
   int num_seqs;
   int num_kv_heads;
   int max_blocks;
@@ -148,6 +164,10 @@ struct TcParams {
   int max_context_len;
   unsigned total_items;
   float scale_log2;
+  // shared-prefix decode: positions below shared_len were attended by the prefix kernel
+  // (partition 0 of every longer context, already in the workspace); this kernel's
+  // partitions start at shared_len and are numbered from 1. 0 = plain decode.
+  int shared_len;
   // fused store (pa_store_decode), else all NULL: row s of new_k / new_v goes to the
   // slot slot_mapping[s], which must be the slot of the sequence's last position
   const uint4* new_k;        // [B, Hkv, D] bf16, 16 vectors per head
@@ -215,13 +235,14 @@ __device__ __forceinline__ unsigned tagged_arrive(unsigned long long* ctr, unsig
 
 // bounded wait that also gives up once another role has given up
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
-                                              volatile int* abort_flag) {
+                                              volatile int* abort_flag,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       flag_error(err, PA_DEV_ERR_TIMEOUT);
       *abort_flag = 1;
       return false;
@@ -272,29 +293,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// 16 e4m3 codes (one uint4, code i in byte i) times a scale -> 16 bf16 values as two
-// uint4 (values 0-7, 8-15; element i in the low half of word i/2 ... as bf16 pairs).
-// e4m3 -> f16 is exact, so code * scale is rounded once (fp32 product, then to bf16).
-// Each step runs over all eight pairs before the next, so the eight chains overlap.
-__device__ __forceinline__ void dequant16(const uint4 raw, float2 scale2, uint4& lo, uint4& hi) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-  __half2_raw h[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    h[i] = __nv_cvt_fp8x2_to_halfraw2(
-        static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu), __NV_E4M3);
-  float2 f[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-#pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = __fmul2_rn(f[i], scale2);
-  uint32_t out[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = pack_bf16x2(f[i].x, f[i].y);
-  lo = make_uint4(out[0], out[1], out[2], out[3]);
-  hi = make_uint4(out[4], out[5], out[6], out[7]);
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -308,12 +306,35 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 
+
+// Two values -> their e4m3 codes (round to nearest even, saturated to +-448), packed
+// with a in the low byte, and the values those codes stand for.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b, float2& back) {
+  const __nv_fp8x2_storage_t c =
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+  back = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return static_cast<uint32_t>(c);
+}
+
+// hi / lo e4m3 terms of two values: hi = e4m3(v), lo = e4m3(lo_scale * (v - hi)),
+// as two packed byte pairs (value a in the low byte of each).
+__device__ __forceinline__ void split_e4m3x2(float a, float b, float lo_scale, uint32_t& hi,
+                                             uint32_t& lo) {
+  float2 h, unused;
+  hi = e4m3x2(a, b, h);
+  lo = e4m3x2((a - h.x) * lo_scale, (b - h.y) * lo_scale, unused);
+}
+
 template <int G, bool F8>
-__global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmSK,
     const __grid_constant__ CUtensorMap tmSV, const TcParams p) {
   static_assert(G >= 1 && G <= NQ, "query heads per kv head");
+  using C = Cfg<F8>;
+  constexpr int NK = C::NK, NV = C::NV, NSC = C::NSC;
+  constexpr int kRegion = C::kRegion, kTileBytes = C::kTileBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -322,8 +343,9 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
   const int lane = tid & 31;
   const int Hq = p.num_kv_heads * G;
   const int bs = 1 << p.bs_log2;
+  const unsigned long long wl = p.wait_ns;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* k_full = bars;                     // [NK] TMA -> issuer
   uint64_t* k_empty = k_full + NK;             // [NK] score MMA done -> producer
   uint64_t* v_full = k_empty + NK;             // [NV] TMA -> issuer (+ softmax)
@@ -340,34 +362,40 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
   uint64_t* epi_empty = epi_full + NO;         // [NO] epilogue read the hand-off
   uint64_t* sched_full = epi_empty + NO;       // [QS] scheduler -> producer
   uint64_t* sched_empty = sched_full + QS;     // [QS] producer done with a queued item
-  uint64_t* kst_full = sched_empty + QS;       // [NK] fp8: codes + scales of K landed
-  uint64_t* vst_full = kst_full + NK;          // [NV] fp8: codes + scales of V landed
-  ItemDesc* sched_desc = reinterpret_cast<ItemDesc*>(smem + kOffSched);
-  int* sched_fb = reinterpret_cast<int*>(smem + kOffSchedFb);
-  ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + kOffDesc);
-  int* ids = reinterpret_cast<int*>(smem + kOffIds);
-  float* red = reinterpret_cast<float*>(smem + kOffRed);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
-  volatile int* conv_stop = reinterpret_cast<volatile int*>(smem + kOffMisc + 32);  // [NK], fp8
+  uint64_t* mma_drain = sched_empty + QS;      // [1] every MMA of the issuer finished
+  uint64_t* ksc_full = mma_drain + 1;          // [NSC] e4m3: K scales of a tile landed
+  uint64_t* ksc_empty = ksc_full + NSC;        // [NSC] e4m3: softmax read them
+  uint64_t* vsc_full = ksc_empty + NSC;        // [NV] e4m3: V scales of a tile landed
+  ItemDesc* sched_desc = reinterpret_cast<ItemDesc*>(smem + C::kOffSched);
+  int* sched_fb = reinterpret_cast<int*>(smem + C::kOffSchedFb);
+  ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + C::kOffDesc);
+  int* ids = reinterpret_cast<int*>(smem + C::kOffIds);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* qscale = reinterpret_cast<float*>(smem + C::kOffQs);  // [QN][NQ] e4m3 q scales
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
+  // e4m3: where a tile's row scales sit (box r / rows, each box on a 128-byte boundary)
+  const int srows = bs < TM ? bs : TM;
+  const int sstride = srows * 4 < 128 ? 128 : srows * 4;
 
   // zero the Q slots and P^T buffers: rows >= G are never written and stay zero
   for (int i = tid; i < (QN * kQBytes + NP * kPBytes) / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(smem + C::kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
-    // fp8: a ring slot is full once every converter warp has written its rows
     for (int i = 0; i < NK; ++i) {
-      mbar_init(&k_full[i], F8 ? conv_warps<G>() : 1);
+      mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&kst_full[i], 1);
-      conv_stop[i] = 0;
     }
     for (int i = 0; i < NV; ++i) {
-      mbar_init(&v_full[i], F8 ? conv_warps<G>() : 1);
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
-      mbar_init(&vst_full[i], 1);
+      if (F8) mbar_init(&vsc_full[i], 1);
+    }
+    for (int i = 0; F8 && i < NSC; ++i) {
+      mbar_init(&ksc_full[i], 1);
+      mbar_init(&ksc_empty[i], 4);
     }
     for (int i = 0; i < QN; ++i) {
       mbar_init(&item_full[i], 1);
@@ -391,11 +419,12 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       mbar_init(&sched_full[i], 1);
       mbar_init(&sched_empty[i], 1);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 5) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -406,28 +435,34 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
   // lane 0 waits, the warp follows its verdict (keeps the warp's control flow uniform)
   auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
     int okw = 0;
-    if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag) ? 1 : 0;
+    if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag, wl) ? 1 : 0;
     return __shfl_sync(0xffffffffu, okw, 0) != 0;
   };
 
   if (warp == 4) {
     // ======================================================== producer warp
     if (lane == 0) {
-      prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
       if (F8) {
         prefetch_tensormap(&tmSK);
         prefetch_tensormap(&tmSV);
+      } else {
+        prefetch_tensormap(&tmQ);
       }
     }
-    const int rows = bs < TM ? bs : TM;
+    const int rows = srows;
     const int nbox = TM / rows;
-    // fp8: each box's scales start on a 128-byte boundary of the slot
-    const int sstride = rows * 4 < 128 ? 128 : rows * 4;
-    int q = 0;       // items taken from the scheduler queue
-    int k = 0;       // items published to the issuer / softmax
-    unsigned j = 0;  // tiles issued
+    int q = 0;        // items taken from the scheduler queue
+    int k = 0;        // items published to the issuer / softmax
+    int kq = 0;       // q loads started (bf16)
+    int npub = 0;     // items published to the item slots (the final stop included)
+    unsigned jk = 0;  // K tiles whose loads were started
+    unsigned jv = 0;  // V tiles whose loads were started
+    auto row_of = [&](const int* idc, int first_blk, int pos) {
+      const int bi = (pos >> p.bs_log2) - first_blk;
+      return (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+    };
     while (true) {
       const int ss = q % QS;
       if (!wwait(&sched_full[ss], (q / QS) & 1)) break;
@@ -441,20 +476,11 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
           descs[slot] = cur;
           mbar_arrive(&item_full[slot]);
         }
-        if (F8) {
-          // the converters follow the tile sequence: mark the next K slot as the end
-          const int ks = j % NK;
-          if (j < NK || wwait(&k_empty[ks], ((j / NK) - 1) & 1)) {
-            if (lane == 0) {
-              conv_stop[ks] = 1;
-              mbar_arrive(&kst_full[ks]);
-            }
-          }
-        }
+        ++npub;
         break;
       }
       const int g = cur.g, t0 = cur.t0, ntiles = cur.ntiles;
-      if (p.slot_mapping != nullptr && cur.p == cur.nparts - 1) {
+      if (!F8 && p.slot_mapping != nullptr && cur.p == cur.nparts - 1) {
         // pa_store_decode: this item reads the sequence's last position, so it writes
         // that position's new row for its kv head first (lanes 0-15: the 16 vectors
         // of K, lanes 16-31: V), then makes the writes visible to its TMA loads.
@@ -481,73 +507,71 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       }
       if (lane == 0) {
         descs[slot] = cur;
-        mbar_arrive_expect_tx(&item_full[slot], 2 * G * 128);
-        uint8_t* qdst = smem + kOffQ + slot * kQBytes;
-        tma_load_3d(qdst, &tmQ, &item_full[slot], 0, g * G, cur.s);
-        tma_load_3d(qdst + kQRegion, &tmQ, &item_full[slot], 64, g * G, cur.s);
+        if (F8) {
+          mbar_arrive(&item_full[slot]);  // the q terms were written by the scheduler
+        } else {
+          mbar_arrive_expect_tx(&item_full[slot], 2 * G * 128);
+          uint8_t* qdst = smem + C::kOffQ + slot * kQBytes;
+          tma_load_3d(qdst, &tmQ, &item_full[slot], 0, g * G, cur.s);
+          tma_load_3d(qdst + kQRegion, &tmQ, &item_full[slot], 64, g * G, cur.s);
+        }
       }
+      if (!F8) kq = k + 1;
+      ++npub;
       bool alive = true;
-      for (int i = 0; i < ntiles; ++i, ++j) {
-        // K of tile j: its slot frees when the score MMA of tile j - NK is done
-        const int ks = j % NK;
-        if (j >= NK && !wwait(&k_empty[ks], ((j / NK) - 1) & 1)) {
+      for (int i = 0; i < ntiles; ++i) {
+        // K of tile jk: its slot frees when the score MMA of tile jk - NK is done
+        const int ks = jk % NK;
+        if (jk >= NK && !wwait(&k_empty[ks], ((jk / NK) - 1) & 1)) {
+          alive = false;
+          break;
+        }
+        const int kl = F8 ? jk % NSC : 0;
+        if (F8 && jk >= NSC && !wwait(&ksc_empty[kl], ((jk / NSC) - 1) & 1)) {
           alive = false;
           break;
         }
         if (lane == 0) {
-          uint8_t* kdst = smem + kOffK + ks * kTileBytes;
-          if (F8) {
-            // codes into the upper half of the slot, scales into the slot's scale area
-            mbar_arrive_expect_tx(&kst_full[ks], kRegion + TM * 4);
-            for (int b = 0; b < nbox; ++b) {
-              const int pos = t0 + i * TM + b * rows;
-              const int bi = (pos >> p.bs_log2) - first_blk;
-              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
-              tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &kst_full[ks], 0, g, row);
-              tma_load_2d(smem + kOffScl + ks * kSclBytes + b * sstride, &tmSK, &kst_full[ks],
+          uint8_t* kdst = smem + C::kOffK + ks * kTileBytes;
+          mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
+          if (F8) mbar_arrive_expect_tx(&ksc_full[kl], TM * 4);
+          for (int b = 0; b < nbox; ++b) {
+            const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
+            if (F8) {
+              tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
+              tma_load_2d(smem + C::kOffScl + kl * kSclBytes + b * sstride, &tmSK, &ksc_full[kl],
                           row, g);
-            }
-          } else {
-            mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
-            for (int b = 0; b < nbox; ++b) {
-              const int pos = t0 + i * TM + b * rows;
-              const int bi = (pos >> p.bs_log2) - first_blk;
-              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+            } else {
               tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
               tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &k_full[ks], 64, g, row);
             }
           }
         }
+        ++jk;
         __syncwarp();
-        // V of tile j: its slot frees when the value MMA of tile j - NV is done
-        const int vs = j % NV;
-        if (j >= NV && !wwait(&v_empty[vs], ((j / NV) - 1) & 1)) {
+        // V of tile jv: its slot frees when the value MMA of tile jv - NV is done
+        const int vs = jv % NV;
+        if (jv >= NV && !wwait(&v_empty[vs], ((jv / NV) - 1) & 1)) {
           alive = false;
           break;
         }
         if (lane == 0) {
-          uint8_t* vdst = smem + kOffV + vs * kTileBytes;
-          if (F8) {
-            mbar_arrive_expect_tx(&vst_full[vs], kRegion + TM * 4);
-            for (int b = 0; b < nbox; ++b) {
-              const int pos = t0 + i * TM + b * rows;
-              const int bi = (pos >> p.bs_log2) - first_blk;
-              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
-              tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &vst_full[vs], 0, g, row);
-              tma_load_2d(smem + kOffScl + (NK + vs) * kSclBytes + b * sstride, &tmSV,
-                          &vst_full[vs], row, g);
-            }
-          } else {
-            mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
-            for (int b = 0; b < nbox; ++b) {
-              const int pos = t0 + i * TM + b * rows;
-              const int bi = (pos >> p.bs_log2) - first_blk;
-              const int row = (bi < kMaxIds ? idc[bi] : 0) * bs + (pos & (bs - 1));
+          uint8_t* vdst = smem + C::kOffV + vs * kTileBytes;
+          mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
+          if (F8) mbar_arrive_expect_tx(&vsc_full[vs], TM * 4);
+          for (int b = 0; b < nbox; ++b) {
+            const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
+            if (F8) {
+              tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
+              tma_load_2d(smem + C::kOffScl + (NSC + vs) * kSclBytes + b * sstride, &tmSV,
+                          &vsc_full[vs], row, g);
+            } else {
               tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
               tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &v_full[vs], 64, g, row);
             }
           }
         }
+        ++jv;
         __syncwarp();
       }
       if (!alive) break;
@@ -555,12 +579,34 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       ++k;
       ++q;
     }
+    // Before the CTA ends, every copy this warp started must have landed. Per slot
+    // only its last load can still be in flight (the one before it was consumed), so
+    // waiting for the last phase of each slot is enough; on the normal path these
+    // completed long ago. Full time limit: these copies always complete.
+    if (lane == 0) {
+      for (unsigned t = jk > static_cast<unsigned>(NK) ? jk - NK : 0; t < jk; ++t)
+        mbar_wait(&k_full[t % NK], (t / NK) & 1, p.err);
+      for (unsigned t = jv > static_cast<unsigned>(NV) ? jv - NV : 0; t < jv; ++t)
+        mbar_wait(&v_full[t % NV], (t / NV) & 1, p.err);
+      if (F8) {
+        for (unsigned t = jk > static_cast<unsigned>(NSC) ? jk - NSC : 0; t < jk; ++t)
+          mbar_wait(&ksc_full[t % NSC], (t / NSC) & 1, p.err);
+        for (unsigned t = jv > static_cast<unsigned>(NV) ? jv - NV : 0; t < jv; ++t)
+          mbar_wait(&vsc_full[t % NV], (t / NV) & 1, p.err);
+      } else {
+        // a q load whose slot took a later item has landed (the slot was handed on only
+        // after the issuer had waited for it); only the others are waited for here
+        for (int t = kq > QN ? kq - QN : 0; t < kq; ++t)
+          if (t + QN >= npub) mbar_wait(&item_full[t % QN], (t / QN) & 1, p.err);
+      }
+    }
   } else if (warp == 10) {
     // ======================================================== scheduler warp
     // Takes items (the CTA's first is its own index, later ones come from the tagged
     // counter), skips empty partitions, reads the context length and the item's
     // block ids, and queues them for the producer QS deep, so none of these dependent
-    // global reads sit on the TMA producer's path.
+    // global reads sit on the TMA producer's path. For e4m3 pools it also writes the
+    // item's q as two e4m3 terms into the item's Q slot.
     int q = 0;
     bool first_take = true;
     while (true) {
@@ -594,8 +640,9 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
           if (lane == 0 && part == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
           ctx = p.max_context_len;
         }
-        if (part * p.partition_size >= ctx) {
-          if (part == 0) {  // empty context: a zero output row
+        const int t0 = p.shared_len + part * p.partition_size;
+        if (t0 >= ctx) {
+          if (part == 0 && p.shared_len == 0) {  // empty context: a zero output row
             for (int i = lane; i < G * HD; i += 32)
               p.out[(static_cast<int64_t>(s) * Hq + g * G) * HD + i] = __float2bfloat16(0.f);
             // and no last position to store a new row at
@@ -604,7 +651,6 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
           }
           continue;
         }
-        const int t0 = part * p.partition_size;
         const int n = min(ctx - t0, p.partition_size);
         const int ntiles = (n + TM - 1) / TM;
         first_blk = t0 >> p.bs_log2;
@@ -621,12 +667,47 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
           }
           idb[i] = id;
         }
-        d.s = s; d.g = g; d.p = part; d.t0 = t0; d.n = n; d.ntiles = ntiles;
-        d.nparts = (ctx + p.partition_size - 1) / p.partition_size;
+        const int shared = p.shared_len > 0 ? 1 : 0;
+        d.s = s; d.g = g; d.p = part + shared; d.t0 = t0; d.n = n; d.ntiles = ntiles;
+        d.nparts = shared + (ctx - p.shared_len + p.partition_size - 1) / p.partition_size;
         d.stop = 0;
         break;
       }
-      __syncwarp();  // the block ids are in shared memory before lane 0 publishes
+      if (F8 && !d.stop) {
+        // q of the item's G heads as e4m3 terms (this scheduler item is the producer's
+        // item q, published to Q slot q % QN): per head s = amax / 448, y = q * 448 /
+        // amax, hi = e4m3(y), lo = e4m3(y - hi). Lane L holds dims 4L..4L+3 and
+        // writes them, 4 bytes per term, into row h of the 128-byte-swizzled slot.
+        const int qs = q % QN;
+        if (q >= QN && !wwait(&item_empty[qs], ((q / QN) - 1) & 1)) {
+          d.stop = 1;
+          d.ntiles = 0;
+        } else {
+          uint8_t* qd = smem + C::kOffQ + qs * kQBytes;
+          const uint2* src = reinterpret_cast<const uint2*>(
+              p.q + (static_cast<int64_t>(d.s) * Hq + d.g * G) * HD);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const uint2 raw = __ldg(src + h * (HD / 4) + lane);
+            const float f0 = bf16lo_to_f32(raw.x), f1 = bf16hi_to_f32(raw.x);
+            const float f2 = bf16lo_to_f32(raw.y), f3 = bf16hi_to_f32(raw.y);
+            float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            float inv = 448.f / amax;
+            if (!(inv <= FLT_MAX)) inv = 0.f;  // all zero (or tiny): codes 0, scale 0
+            uint32_t h01, l01, h23, l23;
+            split_e4m3x2(f0 * inv, f1 * inv, 1.f, h01, l01);
+            split_e4m3x2(f2 * inv, f3 * inv, 1.f, h23, l23);
+            const int off = h * 128 + ((((lane >> 2) ^ h) & 7) << 4) + (lane & 3) * 4;
+            *reinterpret_cast<uint32_t*>(qd + off) = h01 | (h23 << 16);
+            *reinterpret_cast<uint32_t*>(qd + kQRegion + off) = l01 | (l23 << 16);
+            if (lane == 0) qscale[qs * NQ + h] = inv > 0.f ? amax / 448.f : 0.f;
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      __syncwarp();  // the block ids (and q terms) are in shared memory before lane 0 publishes
       if (lane == 0) {
         sched_desc[slot] = d;
         sched_fb[slot] = first_blk;
@@ -638,31 +719,51 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
   } else if (warp == 5) {
     // ======================================================== tensor-core issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(TM, NQ, 0, 0);  // K: K-major, Q^T: K-major
-      constexpr uint32_t idO = idesc_bf16_f32(HD, NQ, 1, 0);  // V^T: MN-major, P^T: K-major
-      const uint32_t sP = smem_u32(smem + kOffP);
+      // bf16: K K-major, Q^T K-major; V^T MN-major, P^T K-major (same for e4m3)
+      constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TM, NQ, 0, 0) : idesc_bf16_f32(TM, NQ, 0, 0);
+      constexpr uint32_t idO = F8 ? idesc_e4m3_f32(HD, NQ, 1, 0) : idesc_bf16_f32(HD, NQ, 1, 0);
+      const uint32_t sP = smem_u32(smem + C::kOffP);
       unsigned j = 0;  // tiles whose score MMA was issued
       // O^T(obuf) += V^T(t) P^T(t); `first` overwrites instead of accumulating
       auto pv = [&](unsigned t, bool first, int obuf, int item) -> bool {
         const int b = t % NP;
         const int vs = t % NV;
-        if (!wait_or_abort(&p_full[b], (t / NP) & 1, p.err, abort_flag) ||
-            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag))
+        if (!wait_or_abort(&p_full[b], (t / NP) & 1, p.err, abort_flag, wl) ||
+            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, wl))
           return false;
         // the first value MMA of an item overwrites O(obuf): the epilogue of the item
         // that used this accumulator NO items ago must have read it
         if (first && item >= NO &&
-            !wait_or_abort(&o_free[obuf], ((item / NO) - 1) & 1, p.err, abort_flag))
+            !wait_or_abort(&o_free[obuf], ((item / NO) - 1) & 1, p.err, abort_flag, wl))
           return false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + kOffV + vs * kTileBytes);
+        const uint32_t sV = smem_u32(smem + C::kOffV + vs * kTileBytes);
         const uint32_t sPt = sP + b * kPBytes;
-        const uint32_t dO = tmem + kTmemO + obuf * 16;
+        const uint32_t dO = tmem + C::kTmemO + obuf * 16;
+        if (F8) {
+          // 32 positions (4 rows of 8-row swizzle atoms) per instruction; the hi term of
+          // P' into O, the lo term into the second accumulator
+          const uint32_t dOlo = tmem + C::kTmemOlo + obuf * 16;
 #pragma unroll
-        for (int kk = 0; kk < TM / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
-          const uint64_t bdesc = smem_desc_sw128(sPt + (kk >> 2) * kQRegion + (kk & 3) * 32, 16, 1024);
-          tc_mma_f16_ss(dO, a, bdesc, idO, (first && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < TM / 32; ++kk) {
+            const uint64_t a = smem_desc_sw128(sV + kk * 32 * 128, kRegion, 1024);
+            tc_mma_f8_ss(dO, a, smem_desc_sw128(sPt + kk * 32, 16, 1024), idO,
+                         (first && kk == 0) ? 0u : 1u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < TM / 32; ++kk) {
+            const uint64_t a = smem_desc_sw128(sV + kk * 32 * 128, kRegion, 1024);
+            tc_mma_f8_ss(dOlo, a, smem_desc_sw128(sPt + kQRegion + kk * 32, 16, 1024), idO,
+                         (first && kk == 0) ? 0u : 1u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < TM / 16; ++kk) {
+            const uint64_t a = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
+            const uint64_t bdesc =
+                smem_desc_sw128(sPt + (kk >> 2) * kQRegion + (kk & 3) * 32, 16, 1024);
+            tc_mma_f16_ss(dO, a, bdesc, idO, (first && kk == 0) ? 0u : 1u);
+          }
         }
         tc_commit(&pv_done[b]);
         tc_commit(&v_empty[vs]);
@@ -672,27 +773,38 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       bool ok = true;
       while (ok) {
         const int slot = k % QN;
-        if (!wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag)) break;
+        if (!wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const ItemDesc d = descs[slot];
         if (d.stop) break;
-        const uint32_t sQ = smem_u32(smem + kOffQ + slot * kQBytes);
+        const uint32_t sQ = smem_u32(smem + C::kOffQ + slot * kQBytes);
         const int obuf = k % NO;
         for (int i = 0; i < d.ntiles; ++i, ++j) {
           const int ks = j % NK;
           const int sb = j % NS;
-          if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag) ||
-              (j >= NS && !wait_or_abort(&s_free[sb], ((j / NS) - 1) & 1, p.err, abort_flag))) {
+          if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, wl) ||
+              (j >= NS && !wait_or_abort(&s_free[sb], ((j / NS) - 1) & 1, p.err, abort_flag, wl))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
+          const uint32_t sK = smem_u32(smem + C::kOffK + ks * kTileBytes);
+          if (F8) {
+            // S^T = K hi^T + K lo^T: 32 head dims (bytes) of each row per instruction
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t ko = (kk >> 2) * kRegion + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * kQRegion + (kk & 3) * 32;
-            tc_mma_f16_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
-                          smem_desc_sw128(sQ + qo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 2 * (HD / 32); ++kk) {
+              const uint32_t ko = (kk & 3) * 32;
+              tc_mma_f8_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
+                           smem_desc_sw128(sQ + (kk >> 2) * kQRegion + ko, 16, 1024), idS,
+                           kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t ko = (kk >> 2) * kRegion + (kk & 3) * 32;
+              const uint32_t qo = (kk >> 2) * kQRegion + (kk & 3) * 32;
+              tc_mma_f16_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
+                            smem_desc_sw128(sQ + qo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&s_full[sb]);
           tc_commit(&k_empty[ks]);                              // K slot reusable
@@ -709,6 +821,9 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
         tc_commit(&o_full[obuf]);  // O(obuf) complete once the MMAs so far are done
         ++k;
       }
+      // every MMA this thread issued has finished before TMEM and shared memory go away
+      tc_commit(mma_drain);
+      mbar_wait(mma_drain, 0, p.err);
     }
   } else if (warp < 4) {
     // ======================================================== softmax warps 0-3
@@ -718,34 +833,41 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
     // at a named barrier.
     const int r = tid;  // position within a tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // e4m3: byte offset of position r's scale within a tile's scale area
+    const int soff = (r / srows) * sstride + (r % srows) * 4;
     int k = 0;
     unsigned j = 0;
     while (true) {
       const int slot = k % QN;
-      bool failed = !wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag);
+      bool failed = !wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl);
       const ItemDesc d = descs[slot];
+      float qsg[G];  // e4m3: the item's per-head q scales
+#pragma unroll
+      for (int h = 0; h < G; ++h) qsg[h] = F8 ? qscale[slot * NQ + h] : 1.f;
       if (bar_or(1, 128, failed)) break;  // every thread has read the descriptor
       if (tid == 0) mbar_arrive(&item_empty[slot]);
       if (d.stop) {
         if (tid == 0) {  // tell the epilogue warps, once they have read slot k % NO
           const int b = k % NO;
-          if (k < NO || wait_or_abort(&epi_empty[b], ((k / NO) - 1) & 1, p.err, abort_flag)) {
-            reinterpret_cast<ItemDesc*>(smem + kOffEpi + b * kEpiBytes)->stop = 1;
+          if (k < NO ||
+              wait_or_abort(&epi_empty[b], ((k / NO) - 1) & 1, p.err, abort_flag, wl)) {
+            reinterpret_cast<ItemDesc*>(smem + C::kOffEpi + b * kEpiBytes)->stop = 1;
             mbar_arrive(&epi_full[b]);
           }
         }
         break;
       }
       const int obuf = k % NO;
-      float m[G], lp[G];
+      float m[G], lp[G], R[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         m[h] = -INFINITY;
         lp[h] = 0.f;
+        R[h] = -INFINITY;  // e4m3: O's reference, unset until a tile has a non-zero V scale
       }
       for (int i = 0; i < d.ntiles; ++i, ++j) {
         const int sb = j % NS;
-        failed |= !wait_or_abort(&s_full[sb], (j / NS) & 1, p.err, abort_flag);
+        failed |= !wait_or_abort(&s_full[sb], (j / NS) & 1, p.err, abort_flag, wl);
         tc_fence_after();
         float sv[16];
         tmem_ld16(tmem + sb * 16 + lane_off, sv);
@@ -754,70 +876,152 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
         const bool valid = i * TM + r < d.n;
+        float x[G];
+        float svr = 0.f;  // e4m3: this position's V scale (0 past the partition)
+        if constexpr (F8) {
+          const int kl = j % NSC;
+          failed |= !wait_or_abort(&ksc_full[kl], (j / NSC) & 1, p.err, abort_flag, wl);
+          const float skr = *reinterpret_cast<const float*>(smem + C::kOffScl + kl * kSclBytes + soff);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ksc_empty[kl]);
+          const int vs = j % NV;
+          failed |= !wait_or_abort(&vsc_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
+          if (valid)
+            svr = *reinterpret_cast<const float*>(smem + C::kOffScl + (NSC + vs) * kSclBytes + soff);
+          const float fr = p.scale_log2 * skr;
+#pragma unroll
+          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * (fr * qsg[h]) : -INFINITY;
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+        }
         // per-head max over the tile: warp shuffles, then across the 4 warps
         float* rb = red + (j & 1) * 4 * NQ;
-        float x[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
           float v = x[h];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) rb[warp * NQ + h] = v;
         }
+        float* svb = red + 3 * 4 * NQ + (j & 1) * 4;  // e4m3: the tile's largest V scale
+        if (F8) {
+          float v = svr;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == 0) svb[warp] = v;
+        }
         named_bar_sync(1, 128);
         bool rescale = false;
         float alpha[G];
+        float pp[G];  // e4m3: P' of this position per head
+        if constexpr (F8) {
+          // bound of P' over the tile: 2^(max x + log2 max s_v - R)
+          const float lsm = lg2_approx(fmaxf(fmaxf(svb[0], svb[1]), fmaxf(svb[2], svb[3])));
+          const float lsv = lg2_approx(svr);  // -inf for s_v = 0 (and past the partition)
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
-          alpha[h] = 1.f;
-          if (i == 0) {
-            m[h] = mx;  // reference max of this item (every tile has a valid position)
-          } else if (mx > m[h] + kRescaleLog2) {
-            alpha[h] = ex2_approx(m[h] - mx);
-            m[h] = mx;
-            rescale = true;
+          for (int h = 0; h < G; ++h) {
+            const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
+            // l's reference (the row sum stays fp32, only its range matters)
+            if (i == 0) {
+              m[h] = mx;
+            } else if (mx > m[h] + kRescaleLog2) {
+              lp[h] *= ex2_approx(m[h] - mx);
+              m[h] = mx;
+            }
+            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
+            lp[h] += pr;
+            // O's reference: set by the first tile with a non-zero V scale (O is exactly
+            // 0 before it), raised when the bound would pass 2^kPBoundLog2
+            alpha[h] = 1.f;
+            const float bnd = mx + lsm;
+            if (R[h] == -INFINITY) {
+              if (bnd > -INFINITY) R[h] = bnd - kPTargetLog2;
+            } else if (bnd > R[h] + kPBoundLog2) {
+              const float rn = bnd - kPTargetLog2;
+              alpha[h] = ex2_approx(R[h] - rn);
+              R[h] = rn;
+              rescale = true;
+            }
+            pp[h] = (valid && R[h] > -INFINITY) ? ex2_approx(x[h] + lsv - R[h]) : 0.f;
           }
-          const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
-          lp[h] = lp[h] * alpha[h] + pr;
-          x[h] = pr;
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
+            alpha[h] = 1.f;
+            if (i == 0) {
+              m[h] = mx;  // reference max of this item (every tile has a valid position)
+            } else if (mx > m[h] + kRescaleLog2) {
+              alpha[h] = ex2_approx(m[h] - mx);
+              m[h] = mx;
+              rescale = true;
+            }
+            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
+            lp[h] = lp[h] * alpha[h] + pr;
+            pp[h] = pr;
+          }
         }
         // this P^T buffer was last read by the value MMA of tile j - NP
         const int pb = j % NP;
-        if (j >= NP) failed |= !wait_or_abort(&pv_done[pb], ((j / NP) - 1) & 1, p.err, abort_flag);
-        uint8_t* pt = smem + kOffP + pb * kPBytes + (r >> 6) * kQRegion;
+        if (j >= NP)
+          failed |= !wait_or_abort(&pv_done[pb], ((j / NP) - 1) & 1, p.err, abort_flag, wl);
+        if constexpr (F8) {
+          // row h of P^T (K-major, 128 positions = 128 bytes, 128-byte swizzle): byte r
+          uint8_t* pt = smem + C::kOffP + pb * kPBytes;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const int chunk = ((r & 63) >> 3) ^ (h & 7);
-          *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + chunk * 16 + (r & 7) * 2) =
-              __float2bfloat16_rn(x[h]);
+          for (int h = 0; h < G; h += 2) {
+            uint32_t hi, lo;
+            split_e4m3x2(pp[h], h + 1 < G ? pp[h + 1] : 0.f, kPLoScale, hi, lo);
+#pragma unroll
+            for (int e = 0; e < 2 && h + e < G; ++e) {
+              const int hh = h + e;
+              const int off = hh * 128 + ((((r >> 4) ^ hh) & 7) << 4) + (r & 15);
+              pt[off] = static_cast<uint8_t>(hi >> (8 * e));
+              pt[kQRegion + off] = static_cast<uint8_t>(lo >> (8 * e));
+            }
+          }
+        } else {
+          uint8_t* pt = smem + C::kOffP + pb * kPBytes + (r >> 6) * kQRegion;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const int chunk = ((r & 63) >> 3) ^ (h & 7);
+            *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + chunk * 16 + (r & 7) * 2) =
+                __float2bfloat16_rn(pp[h]);
+          }
         }
         if (i == d.ntiles - 1 && d.n - i * TM < TM) {
           // V rows past the partition's end may hold anything (even NaN); P is 0 there
           // but 0 * NaN is NaN: clear them before the tensor core reads the tile
           const int vs = j % NV;
-          failed |= !wait_or_abort(&v_full[vs], (j / NV) & 1, p.err, abort_flag);
+          failed |= !wait_or_abort(&v_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
           if (!valid) {
-            uint8_t* v = smem + kOffV + vs * kTileBytes + r * 128;
+            uint8_t* v = smem + C::kOffV + vs * kTileBytes + r * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
+              if (!F8) *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
             }
           }
         }
         if (rescale) {  // uniform across the group: every thread saw the same tile max
           // O holds the value MMAs up to tile j-1: wait for the last of them
           const unsigned t = j - 1;
-          failed |= !wait_or_abort(&pv_done[t % NP], (t / NP) & 1, p.err, abort_flag);
+          failed |= !wait_or_abort(&pv_done[t % NP], (t / NP) & 1, p.err, abort_flag, wl);
           tc_fence_after();
           float o[16];
-          tmem_ld16(tmem + kTmemO + obuf * 16 + lane_off, o);
+          tmem_ld16(tmem + C::kTmemO + obuf * 16 + lane_off, o);
           tc_wait_ld();
 #pragma unroll
           for (int h = 0; h < G; ++h) o[h] *= alpha[h];
-          tmem_st16(tmem + kTmemO + obuf * 16 + lane_off, o);
+          tmem_st16(tmem + C::kTmemO + obuf * 16 + lane_off, o);
+          if (F8) {
+            tmem_ld16(tmem + C::kTmemOlo + obuf * 16 + lane_off, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int h = 0; h < G; ++h) o[h] *= alpha[h];
+            tmem_st16(tmem + C::kTmemOlo + obuf * 16 + lane_off, o);
+          }
           tc_wait_st();
         }
         fence_proxy_async_smem();
@@ -826,7 +1030,8 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
         if (lane == 0) mbar_arrive(&p_full[pb]);
       }
       // hand the item to the epilogue warps: l per head (the per-position shares summed
-      // over the 128 threads) and the reference max; O^T stays in TMEM
+      // over the 128 threads), the reference max and, for e4m3, O's factor 2^(R - m);
+      // O^T stays in TMEM
       float* lb = red + 2 * 4 * NQ;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -838,15 +1043,17 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       named_bar_sync(1, 128);
       if (tid == 0) {
         const int b = k % NO;
-        if (k >= NO) failed |= !wait_or_abort(&epi_empty[b], ((k / NO) - 1) & 1, p.err, abort_flag);
+        if (k >= NO)
+          failed |= !wait_or_abort(&epi_empty[b], ((k / NO) - 1) & 1, p.err, abort_flag, wl);
         if (!failed) {
-          uint8_t* es = smem + kOffEpi + b * kEpiBytes;
+          uint8_t* es = smem + C::kOffEpi + b * kEpiBytes;
           *reinterpret_cast<ItemDesc*>(es) = d;
           float* em = reinterpret_cast<float*>(es + 32);
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             em[h] = m[h];
             em[NQ + h] = lb[h] + lb[NQ + h] + lb[2 * NQ + h] + lb[3 * NQ + h];
+            em[2 * NQ + h] = (F8 && R[h] > -INFINITY) ? ex2_approx(R[h] - m[h]) : (F8 ? 0.f : 1.f);
           }
           mbar_arrive(&epi_full[b]);
         }
@@ -864,23 +1071,32 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
     int k = 0;
     while (true) {
       const int b = k % NO;
-      bool failed = !wait_or_abort(&epi_full[b], (k / NO) & 1, p.err, abort_flag);
-      const uint8_t* es = smem + kOffEpi + b * kEpiBytes;
+      bool failed = !wait_or_abort(&epi_full[b], (k / NO) & 1, p.err, abort_flag, wl);
+      const uint8_t* es = smem + C::kOffEpi + b * kEpiBytes;
       const ItemDesc d = *reinterpret_cast<const ItemDesc*>(es);
-      float m[G], L[G];
+      float m[G], L[G], fac[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         m[h] = reinterpret_cast<const float*>(es + 32)[h];
         L[h] = reinterpret_cast<const float*>(es + 32)[NQ + h];
+        fac[h] = reinterpret_cast<const float*>(es + 32)[2 * NQ + h];
       }
       if (bar_or(2, 128, failed)) break;  // every epilogue thread has read the hand-off
       if (leader) mbar_arrive(&epi_empty[b]);
       if (d.stop) break;
-      failed |= !wait_or_abort(&o_full[b], (k / NO) & 1, p.err, abort_flag);
+      failed |= !wait_or_abort(&o_full[b], (k / NO) & 1, p.err, abort_flag, wl);
       tc_fence_after();
       float o[16];
-      tmem_ld16(tmem + kTmemO + b * 16 + lane_off, o);
-      tc_wait_ld();
+      tmem_ld16(tmem + C::kTmemO + b * 16 + lane_off, o);
+      if (F8) {
+        float olo[16];
+        tmem_ld16(tmem + C::kTmemOlo + b * 16 + lane_off, olo);
+        tc_wait_ld();
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = fmaf(olo[h], 1.f / kPLoScale, o[h]) * fac[h];
+      } else {
+        tc_wait_ld();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[b]);
@@ -907,7 +1123,9 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
           __threadfence();
           bool okc = true;
           const unsigned before = tagged_arrive(p.counters + 1 + row0, p.tag, p.err, &okc);
-          *last_flag = okc && (before == static_cast<unsigned>(d.nparts - 1));
+          // this kernel's partitions of (s, g) (the shared prefix's one came earlier)
+          const int arrivals = d.nparts - (p.shared_len > 0 ? 1 : 0);
+          *last_flag = okc && (before == static_cast<unsigned>(arrivals - 1));
           __threadfence();
         }
         named_bar_sync(2, 128);
@@ -931,88 +1149,12 @@ __global__ void __launch_bounds__(tc_threads<G, F8>(), 1) decode_tc_kernel(
       if (bar_or(2, 128, failed)) break;  // also orders last_flag's reuse
       ++k;
     }
-  } else if (F8) {
-    // ======================================================== converter warps 11..
-    // Follow the tile sequence of the producer; PPR threads (adjacent lanes) share row
-    // r of each K and V tile and dequantise it in place, CPT 16-byte chunks of codes
-    // each. One thread polls the staging barrier while the others sleep in a named
-    // barrier (spinning warps would take issue slots from the MMA and TMA threads);
-    // the vote there also carries abort and end-of-tiles. A row's upper-half bf16
-    // covers only that row's codes, so a warp-level sync orders reads before writes.
-    constexpr int NCT = 32 * conv_warps<G>();
-    constexpr int PPR = NCT / TM;
-    constexpr int CPT = 8 / PPR;
-    const int t = tid - kConvWarp0 * 32;
-    const int r = t / PPR;
-    const int part = t % PPR;
-    const int sw = r & 7;
-    const int rot = r & (CPT - 1);
-    // where the producer put row r's scale: box r / rows, 128-byte aligned boxes
-    const int rows = bs < TM ? bs : TM;
-    const int soff = (r / rows) * (rows * 4 < 128 ? 128 : rows * 4) + (r % rows) * 4;
-    // stop_slot: the K ring slot whose end-of-tiles mark to honour, or -1 (V tiles)
-    auto convert = [&](uint8_t* slot, const uint8_t* scl, uint64_t* staged, unsigned parity,
-                       uint64_t* full, int stop_slot) -> bool {
-      bool quit = false;
-      if (t == 0) {
-        quit = !wait_or_abort(staged, parity, p.err, abort_flag) ||
-               (stop_slot >= 0 && conv_stop[stop_slot] != 0);
-      }
-      if (bar_or(3, NCT, quit)) return false;
-      // the phase is complete (the slot cannot refill before this tile is consumed):
-      // each thread's own test of it orders the TMA's bytes before its reads
-      if (!mbar_try_wait(staged, parity)) flag_error(p.err, PA_DEV_ERR_TIMEOUT);
-      uint4 raw[CPT];
-      // code chunk part * CPT + (c ^ rot) of the row in step c: the 8 threads of a
-      // quarter warp read 8 different 16-byte bank groups (rows are 128 bytes apart)
-      const uint4* src = reinterpret_cast<const uint4*>(slot + kRegion + r * 128);
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) raw[c] = src[part * CPT + (c ^ rot)];
-      const float scv = *reinterpret_cast<const float*>(scl + soff);
-      const float2 sc2 = make_float2(scv, scv);
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        uint4 lo, hi;
-        dequant16(raw[c], sc2, lo, hi);
-        // dims 16k..16k+15 = 16-byte bf16 chunks 2k (lo) and 2k+1 (hi) of the row;
-        // chunk q lies in half q / 8 at position (q % 8) ^ (r % 8) (128-byte swizzle).
-        // The two threads of a row write their chunk pairs in opposite orders, so for
-        // every step the quarter warp's 8 positions are distinct.
-        const int kc = part * CPT + (c ^ rot);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int q = 2 * kc + (h ^ (PPR == 2 ? part : 0));
-          uint4* dst = reinterpret_cast<uint4*>(slot + (q >> 3) * kRegion + r * 128 +
-                                                (((q & 7) ^ sw) << 4));
-          *dst = (q & 1) ? hi : lo;
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(full);
-      return true;
-    };
-    // K(0), V(0), K(1), ... through one call site (keeps the unrolled conversion's
-    // code once in the instruction cache)
-#pragma unroll 1
-    for (unsigned i = 0;; ++i) {
-      const unsigned j = i >> 1;
-      const bool is_v = i & 1;
-      const int rs = is_v ? j % NV : j % NK;
-      const unsigned ph = is_v ? (j / NV) & 1 : (j / NK) & 1;
-      uint8_t* slot = smem + (is_v ? kOffV : kOffK) + rs * kTileBytes;
-      const uint8_t* scl = smem + kOffScl + (is_v ? NK + rs : rs) * kSclBytes;
-      if (!convert(slot, scl, is_v ? &vst_full[rs] : &kst_full[rs], ph,
-                   is_v ? &v_full[rs] : &k_full[rs], is_v ? -1 : rs))
-        break;
-    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -1031,6 +1173,7 @@ unsigned long long next_tag() {
   return v;
 }
 
+
 template <int G, bool F8>
 cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t stream) {
   const int bs = a.cache.block_size;
@@ -1041,14 +1184,14 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
   if (!encode_tensor_map_3d(&tmQ, a.q, HD, a.num_q_heads, a.num_seqs, 64, G, 1, true))
     return cudaErrorInvalidValue;
   if (F8) {
-    // codes [slots][Hkv][D] bytes, one 128-byte row per box row, no swizzle;
-    // scales [Hkv][slots] fp32, a run of `rows` positions of one kv head per box
+    // codes [slots][Hkv][D] bytes, 128-byte rows, 128-byte swizzle (the MMA operand
+    // layout); scales [Hkv][slots] fp32, a run of `rows` positions of one kv head per box
     const uint64_t cd[3] = {HD, hkv, slots};
     const uint32_t cb[3] = {HD, 1, static_cast<uint32_t>(rows)};
     const uint64_t sd[2] = {slots, hkv};
     const uint32_t sb[2] = {static_cast<uint32_t>(rows), 1};
-    if (!encode_tensor_map(&tmK, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, false) ||
-        !encode_tensor_map(&tmV, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, false) ||
+    if (!encode_tensor_map(&tmK, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, true) ||
+        !encode_tensor_map(&tmV, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, cd, cb, true) ||
         !encode_tensor_map(&tmSK, a.k_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, sd, sb, false) ||
         !encode_tensor_map(&tmSV, a.v_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, sd, sb, false))
       return cudaErrorInvalidValue;
@@ -1059,15 +1202,14 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
     tmSK = tmQ;  // unused by the bf16 kernel
     tmSV = tmQ;
   }
-  constexpr int smem_bytes = F8 ? kSmemBytesF8 : kSmemBytes;
+  constexpr int smem_bytes = Cfg<F8>::kSmemBytes;
   cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<G, F8>),
                                           smem_bytes);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  decode_tc_kernel<G, F8><<<grid, tc_threads<G, F8>(), smem_bytes, stream>>>(
-      tmQ, tmK, tmV, tmSK, tmSV, p);
+  decode_tc_kernel<G, F8><<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, tmSK, tmSV, p);
   return cudaGetLastError();
 }
 
@@ -1075,9 +1217,7 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
 
 bool decode_tc_supported(const DecodeLaunch& a) {
   const int G = a.num_q_heads / a.cache.num_kv_heads;
-  // fp8 pools add four or eight converter warps: up to 8 query heads per kv head
-  const bool g_ok = a.fp8 ? (G == 1 || G == 2 || G == 4 || G == 8)
-                          : (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
+  const bool g_ok = G == 1 || G == 2 || G == 4 || G == 8 || G == 16;
   // fp8 scale boxes start at slot index (block id * block size): a multiple of four
   // fp32 (16 bytes) only when the block size is
   const bool bs_ok = !a.fp8 || a.cache.block_size % 4 == 0;
@@ -1089,6 +1229,7 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
                              cudaStream_t stream) {
   TcParams p;
   p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
   p.counters = counters;
@@ -1096,6 +1237,7 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
   p.ws_ml = a.ws_ml;
   p.err = device_error_word();
   p.tag = next_tag();
+  p.wait_ns = wait_limit_ns();
   p.num_seqs = a.num_seqs;
   p.num_kv_heads = a.cache.num_kv_heads;
   p.max_blocks = a.max_blocks_per_seq;
@@ -1104,7 +1246,9 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
   p.partition_size = a.partition_size;
   p.max_parts = a.max_parts;
   p.max_context_len = a.max_context_len;
-  p.total_items = static_cast<unsigned>(a.max_parts) * a.num_seqs * a.cache.num_kv_heads;
+  p.shared_len = a.shared_len;
+  p.total_items = static_cast<unsigned>(a.max_parts - (a.shared_len > 0 ? 1 : 0)) * a.num_seqs *
+                  a.cache.num_kv_heads;
   p.scale_log2 = a.scale * kLog2e;
   p.new_k = static_cast<const uint4*>(a.new_k);
   p.new_v = static_cast<const uint4*>(a.new_v);
@@ -1117,6 +1261,7 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters
       case 2: return launch_tc_t<2, true>(a, p, stream);
       case 4: return launch_tc_t<4, true>(a, p, stream);
       case 8: return launch_tc_t<8, true>(a, p, stream);
+      case 16: return launch_tc_t<16, true>(a, p, stream);
       default: return cudaErrorInvalidValue;
     }
   }

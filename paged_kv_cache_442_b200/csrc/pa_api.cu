@@ -22,7 +22,9 @@ __device__ unsigned g_device_error_word;
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<int> g_debug{0};
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::mutex g_mu;
 int g_sm_count[kMaxDevices] = {0};
 std::set<std::pair<const void*, int>> g_smem_set;  // (kernel, device) already raised
@@ -73,6 +75,8 @@ unsigned* device_error_word() {
   }
   return static_cast<unsigned*>(ptr);
 }
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int sm_count() {
   const int d = current_device();
@@ -260,6 +264,10 @@ const char* pa_status_string(pa_status s) {
 
 void pa_set_debug_checks(int on) { g_debug.store(on ? 1 : 0); }
 
+void pa_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : static_cast<unsigned long long>(ns));
+}
+
 pa_status pa_check_device_errors(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
@@ -359,6 +367,90 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                      workspace, workspace_bytes, stream);
 }
 
+size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t head_dim, int32_t max_context_len,
+                                              int32_t shared_len, int32_t partition_size) {
+  // pa_decode's layout with one more partition (the shared prefix's) in front
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || partition_size <= 0 ||
+      shared_len < 0)
+    return 0;
+  const size_t counters = decode_counter_bytes(num_seqs, num_q_heads);
+  const int64_t rest = max_context_len > shared_len ? max_context_len - shared_len : 0;
+  const int64_t parts = 1 + (rest + partition_size - 1) / partition_size;
+  return counters +
+         static_cast<size_t>(num_seqs) * num_q_heads * parts * (head_dim + 2) * sizeof(float);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, pa_cache_desc cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, float scale, int32_t max_context_len,
+                                  const int32_t* shared_blocks, int32_t shared_len,
+                                  int32_t partition_size, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (shared_len == 0)
+    return pa_decode(out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                     context_lens, num_seqs, num_q_heads, scale, max_context_len, partition_size,
+                     workspace, workspace_bytes, stream);
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+      shared_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache.num_kv_heads || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) >
+          static_cast<int64_t>(max_blocks_per_seq) * cache.block_size ||
+      static_cast<int64_t>(shared_len) >
+          static_cast<int64_t>(max_blocks_per_seq) * cache.block_size)
+    return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache.num_kv_heads;
+  if (cache.head_dim != 128 || (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) ||
+      shared_len % 128 != 0)
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !shared_blocks)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (partition_size < 0 || (partition_size % 128) != 0 || partition_size > 2048)
+    return partition_size < 0 || partition_size % 64 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+  const int32_t rest = max_context_len > shared_len ? max_context_len - shared_len : 0;
+  const int P = partition_size > 0
+                    ? partition_size
+                    : pa_decode_default_partition(num_seqs, cache.num_kv_heads, rest > 0 ? rest : 1);
+  const int64_t parts64 = 1 + (static_cast<int64_t>(rest) + P - 1) / P;
+  if (parts64 * num_seqs * cache.num_kv_heads >= (1ll << 24) - 4096) return PA_ERR_UNSUPPORTED;
+  const size_t need = pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, cache.head_dim,
+                                                             max_context_len, shared_len, P);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+  DecodeLaunch a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cache = cache;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.scale = scale;
+  a.max_context_len = max_context_len;
+  a.partition_size = P;
+  a.max_parts = static_cast<int>(parts64);
+  a.shared_len = shared_len;
+  const size_t cbytes = decode_counter_bytes(num_seqs, num_q_heads);
+  unsigned long long* counters = static_cast<unsigned long long*>(workspace);
+  float* ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
+  a.ws_o = ws;
+  a.ws_ml = ws + static_cast<size_t>(num_seqs) * num_q_heads * a.max_parts * cache.head_dim;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_shared_prefix(a, shared_blocks, shared_len, s);
+  if (e == cudaSuccess && rest > 0) e = launch_decode_tc(a, counters, s);
+  return finish(e, stream);
+}
+
 pa_status pa_store_decode(const void* new_k, const void* new_v, const int32_t* slot_mapping,
                           void* out, const void* q, void* k_cache, void* v_cache,
                           pa_cache_desc cache, const int32_t* block_tables,
@@ -403,11 +495,12 @@ pa_status pa_decode_fp8(void* out, const void* q, const void* k_codes, const voi
                      max_context_len, partition_size, workspace, workspace_bytes, stream);
 }
 
-pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
-                     pa_cache_desc cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
-                     const int32_t* cu_seqlens_q, const int32_t* context_lens, int32_t num_seqs,
-                     int32_t num_q_heads, int32_t total_q, int32_t max_q_len, float scale,
-                     void* stream) {
+namespace {
+pa_status prefill_impl(const StoreRows* store, void* out, const void* q, const void* k_cache,
+                       const void* v_cache, pa_cache_desc cache, const int32_t* block_tables,
+                       int32_t max_blocks_per_seq, const int32_t* cu_seqlens_q,
+                       const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                       int32_t total_q, int32_t max_q_len, float scale, void* stream) {
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || total_q < 0 ||
@@ -420,6 +513,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
   if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_seqlens_q || !context_lens)
     return PA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (store && (!store->new_k || !store->new_v || !store->slot_mapping ||
+                !aligned16(store->new_k) || !aligned16(store->new_v)))
     return PA_ERR_INVALID_ARG;
   PrefillLaunch a;
   a.out = out;
@@ -436,7 +532,35 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
   a.max_q_len = max_q_len;
   a.total_q = total_q;
   a.scale = scale;
+  if (store) {
+    a.new_k = store->new_k;
+    a.new_v = store->new_v;
+    a.slot_mapping = store->slot_mapping;
+  }
   return finish(launch_prefill(a, static_cast<cudaStream_t>(stream)), stream);
+}
+}  // namespace
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     pa_cache_desc cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* cu_seqlens_q, const int32_t* context_lens, int32_t num_seqs,
+                     int32_t num_q_heads, int32_t total_q, int32_t max_q_len, float scale,
+                     void* stream) {
+  return prefill_impl(nullptr, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                      cu_seqlens_q, context_lens, num_seqs, num_q_heads, total_q, max_q_len, scale,
+                      stream);
+}
+
+pa_status pa_store_prefill(const void* new_k, const void* new_v, const int32_t* slot_mapping,
+                           void* out, const void* q, void* k_cache, void* v_cache,
+                           pa_cache_desc cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* cu_seqlens_q,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t total_q, int32_t max_q_len, float scale, void* stream) {
+  const StoreRows rows{new_k, new_v, slot_mapping};
+  return prefill_impl(&rows, out, q, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                      cu_seqlens_q, context_lens, num_seqs, num_q_heads, total_q, max_q_len, scale,
+                      stream);
 }
 
 }  // extern "C"

@@ -18,6 +18,12 @@ constexpr unsigned PA_DEV_ERR_TIMEOUT = 2u;
 // Per-device pointer to the device error word (lives in pa_api.cu).
 unsigned* device_error_word();
 
+// Bound, in ns of %globaltimer, of the waits between the roles of the tensor-core
+// kernels (pa_set_wait_limit_ns; 2 s unless a test shortened it). The waits a CTA
+// makes before it exits, for its own copies and MMAs still in flight, always keep
+// the full 2 s.
+unsigned long long wait_limit_ns();
+
 // Number of SMs of the current device (cached).
 int sm_count();
 
@@ -74,6 +80,9 @@ struct DecodeLaunch {
   bool fp8 = false;
   const float* k_scales = nullptr;
   const float* v_scales = nullptr;
+  // pa_decode_shared_prefix: positions below shared_len are shared by every sequence
+  // (partition 0, attended by launch_shared_prefix); 0 = plain decode
+  int32_t shared_len = 0;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // Stores the new rows of a pa_store_decode call on its own (the paths whose decode
@@ -83,6 +92,10 @@ cudaError_t launch_store_last_rows(const DecodeLaunch& a, cudaStream_t stream);
 // Persistent tcgen05 decode (head dim 128). `counters` is the workspace's counter
 // region: 1 + num_seqs * num_q_heads epoch-tagged 64-bit counters.
 bool decode_tc_supported(const DecodeLaunch& a);
+// The shared prefix of a pa_decode_shared_prefix call, once for all sequences: output
+// rows of contexts inside the prefix, partition-0 partials of the others.
+cudaError_t launch_shared_prefix(const DecodeLaunch& a, const int32_t* shared_blocks,
+                                 int shared_len, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeLaunch& a, unsigned long long* counters,
                              cudaStream_t stream);
 
@@ -107,6 +120,11 @@ struct PrefillLaunch {
   int32_t max_q_len;
   int32_t total_q;  // rows of q/out (cu_seqlens_q[num_seqs]) upper bound for the tensor map
   float scale;
+  // pa_store_prefill: the new rows [total_q, Hkv, D] (read by the attention in place
+  // of the pool) and their slots; all NULL for pa_prefill
+  const void* new_k = nullptr;
+  const void* new_v = nullptr;
+  const int32_t* slot_mapping = nullptr;
 };
 cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
 

@@ -178,10 +178,8 @@ def test_fp8_decode_argument_checks(lib):
     # both scale arrays are required
     assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, NULL, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 32, 128,
                              ws, 1 << 20, NULL) == 1
-    # only the tensor-core path reads e4m3 pools: 16 query heads per kv head, head dim
-    # 64 and partitions that are not a multiple of 128 are valid but not implemented
-    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 32, 0.1, 32, 128,
-                             ws, 1 << 20, NULL) == 2
+    # only the tensor-core path reads e4m3 pools: head dim 64 and partitions that are
+    # not a multiple of 128 are valid but not implemented
     assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, desc(hkv=2, d=64), FAKE, 4, FAKE, 2, 4,
                              0.1, 32, 128, ws, 1 << 20, NULL) == 2
     assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, FAKE, 4, FAKE, 2, 4, 0.1, 32, 192,
