@@ -640,6 +640,12 @@ def main():
                     help="decode steps as pa_store_kvcache + pa_decode instead of pa_store_decode")
     ap.add_argument("--fp8-only", action="store_true",
                     help="print only the decode-batch-64 step over e4m3 pools (one GPU)")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="the configuration's first N sequences only (a small case for "
+                         "profiling; not a headline number)")
+    ap.add_argument("--shared-prefix", action="store_true",
+                    help="decode the workload's shared prefix once for all sequences "
+                         "(pa_decode_shared_prefix; prefix-sharing workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -680,8 +686,9 @@ def main():
                 flush=True)
         return
     # every rank decodes its own batch of the same shape (weak scaling)
-    w = rank_workload(cfg, rank)
-    runner = GpuRunner(w, torch, pa, args.partition_size, args.separate_store)
+    w = rank_workload(cfg, rank, args.num_seqs)
+    shared = cfg.shared_prefix_len if args.shared_prefix else 0
+    runner = GpuRunner(w, torch, pa, args.partition_size, args.separate_store, shared_len=shared)
     flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     sampler = ClockSampler(local_rank)
@@ -704,7 +711,10 @@ def main():
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     if w.kind == "decode":
         kname = ("pa_store_decode (persistent tcgen05 decode; new-row store and split-K merge inside)"
-                 if runner.fused else "pa_decode (persistent tcgen05 decode, split-K merge inside)")
+                 if runner.fused else
+                 "pa_decode_shared_prefix (dense tcgen05 pass over the shared prefix + persistent "
+                 "decode of the rest; time of both launches)" if shared else
+                 "pa_decode (persistent tcgen05 decode, split-K merge inside)")
         roofline = {"bound": "hbm", "kernel": kname,
                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                     "frac": round(achieved / hbm_peak, 3), "peak_source": f"{peak_src} copy bandwidth",
@@ -744,7 +754,8 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+        "config": {"workload": cfg.name + (f" (first {w.num_seqs} sequences)" if args.num_seqs else "")
+                   + (" (shared prefix attended once)" if shared else ""), "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "num_blocks": w.num_blocks,
                    "context_lens": f"{cfg.ctx_dist}[{cfg.ctx_lo},{cfg.ctx_hi}] sum={int(w.context_lens.sum())}",
@@ -804,12 +815,12 @@ def main():
         print(json.dumps(line), flush=True)
 
 
-def rank_workload(cfg, rank):
+def rank_workload(cfg, rank, num_seqs=None):
     """Rank r's batch: the same configuration (shape) drawn from another seed, so the
     ranks decode independent sequences (weak scaling; rank 0's batch is the
-    configuration's own)."""
+    configuration's own). num_seqs keeps the first sequences only (profiling)."""
     from dataclasses import replace
-    return generate(replace(cfg, index=cfg.index + 100 * rank))
+    return generate(replace(cfg, index=cfg.index + 100 * rank), num_seqs=num_seqs)
 
 
 def max_over_ranks(x, dist, torch, device):

@@ -46,9 +46,11 @@
 //     P'_j = 2^(x_j + log2 s_v,j - R), with R a per-item, per-head reference kept so
 //     that P' <= 2^6 (O^T is rescaled when a tile would exceed that, as for the max);
 //     l keeps summing 2^(x_j - m) in fp32, and the output is O^T 2^(R - m) / l;
-//   * q (bf16) becomes two e4m3 terms with one fp32 scale per head, hi = e4m3(q/s)
-//     and lo = e4m3(q/s - hi), written by the scheduler warp; S^T accumulates
-//     K hi^T + K lo^T (about 2^-8 relative error on each q element);
+//   * q (bf16) becomes three e4m3 terms with one fp32 scale per head, hi = e4m3(q/s),
+//     mid = e4m3(q/s - hi), lo = e4m3(q/s - hi - mid), written by the scheduler warp;
+//     S^T accumulates K hi^T + K mid^T + K lo^T (about 2^-13 relative error on a typical
+//     q element: a score error is multiplied by the score's size in the exponent, so
+//     peaked softmaxes need q this exact; K's codes are exact);
 //   * P' becomes hi = e4m3(P') and lo = e4m3(128 (P' - hi)), accumulated into two
 //     O^T accumulators combined as O_hi + O_lo / 128 (about 2^-8 relative on P', and
 //     an absolute floor near 2^-17, so small probabilities keep their precision).
@@ -81,7 +83,7 @@ constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flig
 constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
 constexpr float kRescaleLog2 = 8.f;  // rescale when the max grows by more than this
 constexpr int kQRegion = NQ * 128;           // 16 rows x 128 bytes (2 KB)
-constexpr int kQBytes = 2 * kQRegion;        // bf16: two 64-dim halves; e4m3: hi, lo terms
+constexpr int kQTerms = 3;                   // e4m3: q as hi + mid + lo terms
 constexpr int kPBytes = 2 * kQRegion;        // bf16: P^T 16 x 128; e4m3: hi, lo terms
 constexpr int kMaxIds = 2048 / 16 + 2;       // block ids of one item (partition <= 2048)
 constexpr int kSclBytes = 1024;              // e4m3: one tile's row scales (<= 8 boxes)
@@ -105,6 +107,7 @@ struct Cfg {
   static constexpr int NK = F8 ? 5 : 3;  // K ring (a slot frees when its score MMA is done)
   static constexpr int NV = F8 ? 6 : 3;  // V ring (a slot frees when its value MMA is done)
   static constexpr int NSC = F8 ? 8 : 1;  // e4m3: K-scale ring (freed by the softmax); unused for bf16
+  static constexpr int kQBytes = (F8 ? kQTerms : 2) * kQRegion;  // bf16: two 64-dim halves
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + NK * kTileBytes;
   static constexpr int kOffQ = kOffV + NV * kTileBytes;
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   const int sstride = srows * 4 < 128 ? 128 : srows * 4;
 
   // zero the Q slots and P^T buffers: rows >= G are never written and stay zero
-  for (int i = tid; i < (QN * kQBytes + NP * kPBytes) / 16; i += blockDim.x)
+  for (int i = tid; i < (QN * C::kQBytes + NP * kPBytes) / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + C::kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
@@ -431,6 +434,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp == 4 && lane == 0) {  // the tensor maps are kernel parameters
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    if (F8) {
+      prefetch_tensormap(&tmSK);
+      prefetch_tensormap(&tmSV);
+    } else {
+      prefetch_tensormap(&tmQ);
+    }
+  }
+  // launched as a programmatic dependent: everything above overlapped the previous
+  // kernel's tail; global memory is read only from here on
+  grid_dependency_wait();
+  allow_dependent_launch();
 
   // lane 0 waits, the warp follows its verdict (keeps the warp's control flow uniform)
   auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
@@ -441,16 +458,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
 
   if (warp == 4) {
     // ======================================================== producer warp
-    if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      if (F8) {
-        prefetch_tensormap(&tmSK);
-        prefetch_tensormap(&tmSV);
-      } else {
-        prefetch_tensormap(&tmQ);
-      }
-    }
     const int rows = srows;
     const int nbox = TM / rows;
     int q = 0;        // items taken from the scheduler queue
@@ -511,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           mbar_arrive(&item_full[slot]);  // the q terms were written by the scheduler
         } else {
           mbar_arrive_expect_tx(&item_full[slot], 2 * G * 128);
-          uint8_t* qdst = smem + C::kOffQ + slot * kQBytes;
+          uint8_t* qdst = smem + C::kOffQ + slot * C::kQBytes;
           tma_load_3d(qdst, &tmQ, &item_full[slot], 0, g * G, cur.s);
           tma_load_3d(qdst + kQRegion, &tmQ, &item_full[slot], 64, g * G, cur.s);
         }
@@ -683,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           d.stop = 1;
           d.ntiles = 0;
         } else {
-          uint8_t* qd = smem + C::kOffQ + qs * kQBytes;
+          uint8_t* qd = smem + C::kOffQ + qs * C::kQBytes;
           const uint2* src = reinterpret_cast<const uint2*>(
               p.q + (static_cast<int64_t>(d.s) * Hq + d.g * G) * HD);
 #pragma unroll
@@ -696,12 +703,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             float inv = 448.f / amax;
             if (!(inv <= FLT_MAX)) inv = 0.f;  // all zero (or tiny): codes 0, scale 0
-            uint32_t h01, l01, h23, l23;
-            split_e4m3x2(f0 * inv, f1 * inv, 1.f, h01, l01);
-            split_e4m3x2(f2 * inv, f3 * inv, 1.f, h23, l23);
+            // three terms: each is the e4m3 rounding of what the terms before it left
+            float y[4] = {f0 * inv, f1 * inv, f2 * inv, f3 * inv};
             const int off = h * 128 + ((((lane >> 2) ^ h) & 7) << 4) + (lane & 3) * 4;
-            *reinterpret_cast<uint32_t*>(qd + off) = h01 | (h23 << 16);
-            *reinterpret_cast<uint32_t*>(qd + kQRegion + off) = l01 | (l23 << 16);
+#pragma unroll
+            for (int term = 0; term < kQTerms; ++term) {
+              float2 b01, b23;
+              const uint32_t c01 = e4m3x2(y[0], y[1], b01);
+              const uint32_t c23 = e4m3x2(y[2], y[3], b23);
+              *reinterpret_cast<uint32_t*>(qd + term * kQRegion + off) = c01 | (c23 << 16);
+              y[0] -= b01.x;
+              y[1] -= b01.y;
+              y[2] -= b23.x;
+              y[3] -= b23.y;
+            }
             if (lane == 0) qscale[qs * NQ + h] = inv > 0.f ? amax / 448.f : 0.f;
           }
           fence_proxy_async_smem();
@@ -776,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (!wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const ItemDesc d = descs[slot];
         if (d.stop) break;
-        const uint32_t sQ = smem_u32(smem + C::kOffQ + slot * kQBytes);
+        const uint32_t sQ = smem_u32(smem + C::kOffQ + slot * C::kQBytes);
         const int obuf = k % NO;
         for (int i = 0; i < d.ntiles; ++i, ++j) {
           const int ks = j % NK;
@@ -789,9 +804,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           tc_fence_after();
           const uint32_t sK = smem_u32(smem + C::kOffK + ks * kTileBytes);
           if (F8) {
-            // S^T = K hi^T + K lo^T: 32 head dims (bytes) of each row per instruction
+            // S^T = K hi^T + K mid^T + K lo^T: 32 head dims (bytes) of each row per
+            // instruction
 #pragma unroll
-            for (int kk = 0; kk < 2 * (HD / 32); ++kk) {
+            for (int kk = 0; kk < kQTerms * (HD / 32); ++kk) {
               const uint32_t ko = (kk & 3) * 32;
               tc_mma_f8_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
                            smem_desc_sw128(sQ + (kk >> 2) * kQRegion + ko, 16, 1024), idS,
@@ -1209,8 +1225,19 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  decode_tc_kernel<G, F8><<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, tmSK, tmSV, p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the CTAs' set-up (barriers, tensor memory, tensor
+  // map prefetch) overlaps the tail of the previous kernel in the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8>, tmQ, tmK, tmV, tmSK, tmSV, p);
 }
 
 }  // namespace

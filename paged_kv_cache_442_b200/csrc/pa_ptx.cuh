@@ -125,6 +125,19 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// ----------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream still runs; it must
+// wait here before it reads anything that kernel (or an earlier one) wrote.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel of the stream (if launched as a dependent) start its prologue.
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -315,6 +328,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for two values on the FMA pipe, to take part of the softmax's exponentials off
+// the special-function unit. Cody-Waite range reduction: n = round(x) (adding 1.5 * 2^23
+// leaves n in the low bits of the sum), f = x - n in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial fitted to 2^f over that interval, near-minimax in relative error
+// (iteratively reweighted least squares at Chebyshev nodes; max relative error 7.5e-5,
+// i.e. 2^-13.7, well below the bf16 rounding the probabilities get); then n is added to
+// the exponent bits (the constant's own bits vanish in the shift by 23). Inputs are
+// clamped to [-126, +inf): results below 2^-126 are tiny positive values, not 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.055171654f;
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  const int ex = (__float_as_int(t.x) << 23) + __float_as_int(p.x);
+  const int ey = (__float_as_int(t.y) << 23) + __float_as_int(p.y);
+  return make_float2(__int_as_float(ex), __int_as_float(ey));
 }
 
 // log2 (approximate; subnormal inputs are not flushed, 0 gives -inf)
