@@ -209,6 +209,8 @@ class GpuRunner:
         elif w.kind == "decode":
             self.ws, self.P = pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads,
                                                   w.head_dim, w.max_context_len, partition_size)
+        tc = False
+        if w.kind == "decode":
             # kernels one pa_decode launches: the persistent tcgen05 kernel merges its
             # partitions itself (head dim 128, partition a multiple of 128 up to 2048);
             # the CUDA-core kernel adds a reduce launch when the context is split
@@ -465,7 +467,7 @@ class PackedInputs:
                   ("bt", runner.block_tables)]
         self.layout, off = {}, 0
         for name, t in pieces:
-            if t is None:
+            if t is None or t.numel() == 0:
                 continue
             n = t.numel() * t.element_size()
             self.layout[name] = (off, n, t.dtype, tuple(t.shape))
@@ -473,7 +475,7 @@ class PackedInputs:
         self.nbytes = off
         self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
         for name, t in pieces:
-            if t is not None:
+            if t is not None and name in self.layout:
                 o, n, _, _ = self.layout[name]
                 self.host[o:o + n].copy_(t.contiguous().view(torch.uint8).view(-1).cpu())
         self.torch = torch
@@ -502,8 +504,9 @@ def time_e2e(runner, torch, steps, warmup):
 
     def one(views, dout, hout, copy_stream=None):
         d = views
-        runner.store(d.get("k"), d.get("v"), d["slots"])
-        runner.attend(d["q"], d["ctx"], d["bt"], dout, d.get("k"), d.get("v"), d["slots"])
+        slots = d.get("slots", runner.new_slots)   # an empty slot list is not copied
+        runner.store(d.get("k"), d.get("v"), slots)
+        runner.attend(d["q"], d["ctx"], d["bt"], dout, d.get("k"), d.get("v"), slots)
 
     def serial():
         d_in.copy_(pk.host, non_blocking=True)

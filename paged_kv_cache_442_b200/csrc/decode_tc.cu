@@ -122,7 +122,7 @@ struct Cfg {
   static constexpr int kOffEpi = align_up(kOffDesc + QN * 32, 16);            // [NO] hand-offs
   static constexpr int kOffBar = align_up(kOffEpi + NO * kEpiBytes, 16);
   static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS +
-                                  1 + (F8 ? 2 * NSC + NV : 0);
+                                  1 + (F8 ? 2 * NSC + NV + QN : 0);
   static constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
   // e4m3: the K-scale ring [NSC] and each V slot's scales [NV], 1 KB each
   static constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   uint64_t* ksc_full = mma_drain + 1;          // [NSC] e4m3: K scales of a tile landed
   uint64_t* ksc_empty = ksc_full + NSC;        // [NSC] e4m3: softmax read them
   uint64_t* vsc_full = ksc_empty + NSC;        // [NV] e4m3: V scales of a tile landed
+  uint64_t* q_ready = vsc_full + NV;           // [QN] e4m3: the item's q terms written
   ItemDesc* sched_desc = reinterpret_cast<ItemDesc*>(smem + C::kOffSched);
   int* sched_fb = reinterpret_cast<int*>(smem + C::kOffSchedFb);
   ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + C::kOffDesc);
@@ -400,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       mbar_init(&ksc_full[i], 1);
       mbar_init(&ksc_empty[i], 4);
     }
+    for (int i = 0; F8 && i < QN; ++i) mbar_init(&q_ready[i], 1);
     for (int i = 0; i < QN; ++i) {
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], 2);
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp == 4 && lane == 0) {  // the tensor maps are kernel parameters
+  if (warp == 4 && lane == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     if (F8) {
@@ -444,10 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       prefetch_tensormap(&tmQ);
     }
   }
-  // launched as a programmatic dependent: everything above overlapped the previous
-  // kernel's tail; global memory is read only from here on
-  grid_dependency_wait();
-  allow_dependent_launch();
 
   // lane 0 waits, the warp follows its verdict (keeps the warp's control flow uniform)
   auto wwait = [&](uint64_t* bar, unsigned parity) -> bool {
@@ -680,55 +678,54 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         d.stop = 0;
         break;
       }
-      if (F8 && !d.stop) {
-        // q of the item's G heads as e4m3 terms (this scheduler item is the producer's
-        // item q, published to Q slot q % QN): per head s = amax / 448, y = q * 448 /
-        // amax, hi = e4m3(y), lo = e4m3(y - hi). Lane L holds dims 4L..4L+3 and
-        // writes them, 4 bytes per term, into row h of the 128-byte-swizzled slot.
-        const int qs = q % QN;
-        if (q >= QN && !wwait(&item_empty[qs], ((q / QN) - 1) & 1)) {
-          d.stop = 1;
-          d.ntiles = 0;
-        } else {
-          uint8_t* qd = smem + C::kOffQ + qs * C::kQBytes;
-          const uint2* src = reinterpret_cast<const uint2*>(
-              p.q + (static_cast<int64_t>(d.s) * Hq + d.g * G) * HD);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const uint2 raw = __ldg(src + h * (HD / 4) + lane);
-            const float f0 = bf16lo_to_f32(raw.x), f1 = bf16hi_to_f32(raw.x);
-            const float f2 = bf16lo_to_f32(raw.y), f3 = bf16hi_to_f32(raw.y);
-            float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            float inv = 448.f / amax;
-            if (!(inv <= FLT_MAX)) inv = 0.f;  // all zero (or tiny): codes 0, scale 0
-            // three terms: each is the e4m3 rounding of what the terms before it left
-            float y[4] = {f0 * inv, f1 * inv, f2 * inv, f3 * inv};
-            const int off = h * 128 + ((((lane >> 2) ^ h) & 7) << 4) + (lane & 3) * 4;
-#pragma unroll
-            for (int term = 0; term < kQTerms; ++term) {
-              float2 b01, b23;
-              const uint32_t c01 = e4m3x2(y[0], y[1], b01);
-              const uint32_t c23 = e4m3x2(y[2], y[3], b23);
-              *reinterpret_cast<uint32_t*>(qd + term * kQRegion + off) = c01 | (c23 << 16);
-              y[0] -= b01.x;
-              y[1] -= b01.y;
-              y[2] -= b23.x;
-              y[3] -= b23.y;
-            }
-            if (lane == 0) qscale[qs * NQ + h] = inv > 0.f ? amax / 448.f : 0.f;
-          }
-          fence_proxy_async_smem();
-        }
-      }
-      __syncwarp();  // the block ids (and q terms) are in shared memory before lane 0 publishes
+      __syncwarp();  // the block ids are in shared memory before lane 0 publishes
       if (lane == 0) {
         sched_desc[slot] = d;
         sched_fb[slot] = first_blk;
         mbar_arrive(&sched_full[slot]);
       }
       if (d.stop) break;
+      if (F8) {
+        // q of the item's G heads as e4m3 terms, after the item is published (the
+        // producer starts its tiles meanwhile); this scheduler item is the producer's
+        // item q, in Q slot q % QN, whose previous item's score MMAs must be done. Per
+        // head s = amax / 448, y = q * 448 / amax; lane L holds dims 4L..4L+3 and writes
+        // them, 4 bytes per term, into row h of the 128-byte-swizzled slot.
+        const int qs = q % QN;
+        if (q >= QN && !wwait(&item_empty[qs], ((q / QN) - 1) & 1)) break;
+        uint8_t* qd = smem + C::kOffQ + qs * C::kQBytes;
+        const uint2* src = reinterpret_cast<const uint2*>(
+            p.q + (static_cast<int64_t>(d.s) * Hq + d.g * G) * HD);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const uint2 raw = __ldg(src + h * (HD / 4) + lane);
+          const float f0 = bf16lo_to_f32(raw.x), f1 = bf16hi_to_f32(raw.x);
+          const float f2 = bf16lo_to_f32(raw.y), f3 = bf16hi_to_f32(raw.y);
+          float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          float inv = 448.f / amax;
+          if (!(inv <= FLT_MAX)) inv = 0.f;  // all zero (or tiny): codes 0, scale 0
+          // three terms: each is the e4m3 rounding of what the terms before it left
+          float y[4] = {f0 * inv, f1 * inv, f2 * inv, f3 * inv};
+          const int off = h * 128 + ((((lane >> 2) ^ h) & 7) << 4) + (lane & 3) * 4;
+#pragma unroll
+          for (int term = 0; term < kQTerms; ++term) {
+            float2 b01, b23;
+            const uint32_t c01 = e4m3x2(y[0], y[1], b01);
+            const uint32_t c23 = e4m3x2(y[2], y[3], b23);
+            *reinterpret_cast<uint32_t*>(qd + term * kQRegion + off) = c01 | (c23 << 16);
+            y[0] -= b01.x;
+            y[1] -= b01.y;
+            y[2] -= b23.x;
+            y[3] -= b23.y;
+          }
+          if (lane == 0) qscale[qs * NQ + h] = inv > 0.f ? amax / 448.f : 0.f;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready[qs]);
+      }
       ++q;
     }
   } else if (warp == 5) {
@@ -791,6 +788,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (!wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const ItemDesc d = descs[slot];
         if (d.stop) break;
+        // e4m3: the scheduler writes the item's q terms after publishing the item
+        if (F8 && !wait_or_abort(&q_ready[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const uint32_t sQ = smem_u32(smem + C::kOffQ + slot * C::kQBytes);
         const int obuf = k % NO;
         for (int i = 0; i < d.ntiles; ++i, ++j) {
@@ -857,7 +856,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       const int slot = k % QN;
       bool failed = !wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl);
       const ItemDesc d = descs[slot];
-      float qsg[G];  // e4m3: the item's per-head q scales
+      // e4m3: the item's per-head q scales, written with its q terms
+      if (F8 && !d.stop)
+        failed |= !wait_or_abort(&q_ready[slot], (k / QN) & 1, p.err, abort_flag, wl);
+      float qsg[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) qsg[h] = F8 ? qscale[slot * NQ + h] : 1.f;
       if (bar_or(1, 128, failed)) break;  // every thread has read the descriptor
@@ -1146,17 +1148,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         }
         named_bar_sync(2, 128);
         if (*last_flag) {
-          // this CTA completed the last partition of (s, g): merge all of them
+          // this CTA completed the last partition of (s, g): merge all of them. The
+          // partials are read eight partitions at a time with independent loads (one
+          // round trip per chunk, not one per partition)
+          constexpr int CH = 8;
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const int64_t base = (row0 + h) * p.max_parts;
+            const int np = d.nparts;
             float M = -INFINITY;
-            for (int q = 0; q < d.nparts; ++q) M = fmaxf(M, __ldcg(p.ws_ml + (base + q) * 2));
+            for (int q0 = 0; q0 < np; q0 += CH) {
+              float mm[CH];
+#pragma unroll
+              for (int i = 0; i < CH; ++i)
+                mm[i] = q0 + i < np ? __ldcg(p.ws_ml + (base + q0 + i) * 2) : -INFINITY;
+#pragma unroll
+              for (int i = 0; i < CH; ++i) M = fmaxf(M, mm[i]);
+            }
             float Ls = 0.f, acc = 0.f;
-            for (int q = 0; q < d.nparts; ++q) {
-              const float f = ex2_approx(__ldcg(p.ws_ml + (base + q) * 2) - M);
-              Ls += __ldcg(p.ws_ml + (base + q) * 2 + 1) * f;
-              acc += __ldcg(p.ws_o + (base + q) * HD + dl) * f;
+            for (int q0 = 0; q0 < np; q0 += CH) {
+              float2 ml[CH];
+              float oo[CH];
+#pragma unroll
+              for (int i = 0; i < CH; ++i) {
+                const bool in = q0 + i < np;
+                ml[i] = in ? __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + base + q0 + i)
+                           : make_float2(-INFINITY, 0.f);
+                oo[i] = in ? __ldcg(p.ws_o + (base + q0 + i) * HD + dl) : 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < CH; ++i) {
+                const float f = ex2_approx(ml[i].x - M);
+                Ls += ml[i].y * f;
+                acc += oo[i] * f;
+              }
             }
             p.out[(row0 + h) * HD + dl] = __float2bfloat16_rn(acc / Ls);
           }
@@ -1225,19 +1250,8 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  // programmatic dependent launch: the CTAs' set-up (barriers, tensor memory, tensor
-  // map prefetch) overlaps the tail of the previous kernel in the stream
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem_bytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8>, tmQ, tmK, tmV, tmSK, tmSV, p);
+  decode_tc_kernel<G, F8><<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, tmSK, tmSV, p);
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -125,19 +125,6 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// ----------------------------------------------------------------- dependent launch
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start while the previous kernel of the stream still runs; it must
-// wait here before it reads anything that kernel (or an earlier one) wrote.
-__device__ __forceinline__ void grid_dependency_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-// Lets the next kernel of the stream (if launched as a dependent) start its prologue.
-__device__ __forceinline__ void allow_dependent_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
