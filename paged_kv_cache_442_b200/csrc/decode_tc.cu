@@ -749,33 +749,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             !wait_or_abort(&o_free[obuf], ((item / NO) - 1) & 1, p.err, abort_flag, wl))
           return false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + C::kOffV + vs * kTileBytes);
-        const uint32_t sPt = sP + b * kPBytes;
+        // one descriptor per operand, stepped by constant offsets (see desc_advance)
+        const uint64_t aV = smem_desc_sw128(smem_u32(smem + C::kOffV + vs * kTileBytes),
+                                            kRegion, 1024);
+        const uint64_t bP = smem_desc_sw128(sP + b * kPBytes, 16, 1024);
         const uint32_t dO = tmem + C::kTmemO + obuf * 16;
         if (F8) {
           // 32 positions (4 rows of 8-row swizzle atoms) per instruction; the hi term of
           // P' into O, the lo term into the second accumulator
           const uint32_t dOlo = tmem + C::kTmemOlo + obuf * 16;
 #pragma unroll
-          for (int kk = 0; kk < TM / 32; ++kk) {
-            const uint64_t a = smem_desc_sw128(sV + kk * 32 * 128, kRegion, 1024);
-            tc_mma_f8_ss(dO, a, smem_desc_sw128(sPt + kk * 32, 16, 1024), idO,
+          for (int kk = 0; kk < TM / 32; ++kk)
+            tc_mma_f8_ss(dO, desc_advance(aV, kk * 32 * 128), desc_advance(bP, kk * 32), idO,
                          (first && kk == 0) ? 0u : 1u);
-          }
 #pragma unroll
-          for (int kk = 0; kk < TM / 32; ++kk) {
-            const uint64_t a = smem_desc_sw128(sV + kk * 32 * 128, kRegion, 1024);
-            tc_mma_f8_ss(dOlo, a, smem_desc_sw128(sPt + kQRegion + kk * 32, 16, 1024), idO,
-                         (first && kk == 0) ? 0u : 1u);
-          }
+          for (int kk = 0; kk < TM / 32; ++kk)
+            tc_mma_f8_ss(dOlo, desc_advance(aV, kk * 32 * 128),
+                         desc_advance(bP, kQRegion + kk * 32), idO, (first && kk == 0) ? 0u : 1u);
         } else {
 #pragma unroll
-          for (int kk = 0; kk < TM / 16; ++kk) {
-            const uint64_t a = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
-            const uint64_t bdesc =
-                smem_desc_sw128(sPt + (kk >> 2) * kQRegion + (kk & 3) * 32, 16, 1024);
-            tc_mma_f16_ss(dO, a, bdesc, idO, (first && kk == 0) ? 0u : 1u);
-          }
+          for (int kk = 0; kk < TM / 16; ++kk)
+            tc_mma_f16_ss(dO, desc_advance(aV, kk * 16 * 128),
+                          desc_advance(bP, (kk >> 2) * kQRegion + (kk & 3) * 32), idO,
+                          (first && kk == 0) ? 0u : 1u);
         }
         tc_commit(&pv_done[b]);
         tc_commit(&v_empty[vs]);
@@ -801,25 +797,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             break;
           }
           tc_fence_after();
-          const uint32_t sK = smem_u32(smem + C::kOffK + ks * kTileBytes);
+          const uint64_t aK = smem_desc_sw128(smem_u32(smem + C::kOffK + ks * kTileBytes), 16, 1024);
+          const uint64_t bQ = smem_desc_sw128(sQ, 16, 1024);
           if (F8) {
             // S^T = K hi^T + K mid^T + K lo^T: 32 head dims (bytes) of each row per
             // instruction
 #pragma unroll
-            for (int kk = 0; kk < kQTerms * (HD / 32); ++kk) {
-              const uint32_t ko = (kk & 3) * 32;
-              tc_mma_f8_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
-                           smem_desc_sw128(sQ + (kk >> 2) * kQRegion + ko, 16, 1024), idS,
+            for (int kk = 0; kk < kQTerms * (HD / 32); ++kk)
+              tc_mma_f8_ss(tmem + sb * 16, desc_advance(aK, (kk & 3) * 32),
+                           desc_advance(bQ, (kk >> 2) * kQRegion + (kk & 3) * 32), idS,
                            kk > 0 ? 1u : 0u);
-            }
           } else {
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
-              const uint32_t ko = (kk >> 2) * kRegion + (kk & 3) * 32;
-              const uint32_t qo = (kk >> 2) * kQRegion + (kk & 3) * 32;
-              tc_mma_f16_ss(tmem + sb * 16, smem_desc_sw128(sK + ko, 16, 1024),
-                            smem_desc_sw128(sQ + qo, 16, 1024), idS, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < HD / 16; ++kk)
+              tc_mma_f16_ss(tmem + sb * 16, desc_advance(aK, (kk >> 2) * kRegion + (kk & 3) * 32),
+                            desc_advance(bQ, (kk >> 2) * kQRegion + (kk & 3) * 32), idS,
+                            kk > 0 ? 1u : 0u);
           }
           tc_commit(&s_full[sb]);
           tc_commit(&k_empty[ks]);                              // K slot reusable

@@ -289,6 +289,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of the same operand `bytes` further on (a 16-byte multiple): only the
+// start-address field (bits 0-13, in 16-byte units) changes, and it does not carry
+// into the next field for shared-memory addresses below 256 KB. Used to step through
+// the K slices of one operand without rebuilding its descriptor for every MMA.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   15 A major (0 = K, 1 = MN), 16 B major, 17-22 N >> 3, 24-28 M >> 4.

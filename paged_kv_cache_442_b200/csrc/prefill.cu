@@ -339,13 +339,14 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
         if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns))
           return false;
         tc_fence_after();
-        const uint32_t sQ = smem_u32(smem + kOffQ + u * kTileBytes);
-        const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
+        // one descriptor per operand, stepped by constant offsets (see desc_advance)
+        const uint64_t aQ = smem_desc_sw128(smem_u32(smem + kOffQ + u * kTileBytes), 16, 1024);
+        const uint64_t bK = smem_desc_sw128(smem_u32(smem + kOffK + ks * kTileBytes), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-          tc_mma_f16_ss(tmem + u * 128, smem_desc_sw128(sQ + off, 16, 1024),
-                        smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          tc_mma_f16_ss(tmem + u * 128, desc_advance(aQ, off), desc_advance(bK, off), idS,
+                        kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[u]);
         if (u == 1 || j >= nt1) tc_commit(&k_empty[ks]);
@@ -359,14 +360,11 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
           return false;
         tc_fence_after();
         const uint32_t tP = tmem + u * 128;
-        const uint32_t sV = smem_u32(smem + kOffV + vs * kTileBytes);
+        const uint64_t bV = smem_desc_sw128(smem_u32(smem + kOffV + vs * kTileBytes), kRegion, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // 16 kv positions per step = 8 packed columns of P
-          const uint64_t bd = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
-          tc_mma_f16_ts(tmem + kTmemO + u * 128, tP + kk * 8, bd, idO,
+        for (int kk = 0; kk < BN / 16; ++kk)  // 16 kv positions per step = 8 packed columns of P
+          tc_mma_f16_ts(tmem + kTmemO + u * 128, tP + kk * 8, desc_advance(bV, kk * 16 * 128), idO,
                         (t > 0 || kk > 0) ? 1u : 0u);
-        }
         tc_commit(&pv_done[u]);
         if (u == 1 || t >= nt1) tc_commit(&v_empty[vs]);
         return true;

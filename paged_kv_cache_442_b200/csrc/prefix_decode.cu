@@ -15,10 +15,15 @@
 // (m, l, o) of partition 0 of the split-K decode (the same record and reference as the
 // decode kernel's partitions), which the persistent decode over the remaining
 // positions merges in.
-// Roles (192 threads): warps 0-3 softmax + output, warp 4 TMA producer (Q once,
-// K and V of the shared blocks, two-deep rings),
-// warp 5 TMEM owner and MMA issuer. The producer warp also checks that every
-// sequence of the CTA's rows has the same block ids over the shared prefix.
+// Each CTA takes two such tiles of 128 query rows (units 0 and 1, consecutive rows of
+// one kv head) that read the same shared tiles, and the tensor core alternates between
+// them: issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so one unit's softmax runs
+// while the other unit's products execute (P_u is written over S_u in TMEM, and
+// S_u(j+1) done implies PV_u(j) done).
+// Roles (320 threads): warps 0-3 / 4-7 softmax + output of unit 0 / 1, warp 8 TMA
+// producer (both Q tiles, then K and V of the shared blocks in two-deep rings),
+// warp 9 TMEM owner (all 512 columns: S_0/P_0, S_1/P_1, O_0, O_1) and MMA issuer. The
+// producer warp also checks every sequence of the CTA's rows against the shared blocks.
 #include <cuda_bf16.h>
 
 #include "pa_internal.h"
@@ -30,18 +35,18 @@ namespace {
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // shared positions per tile
 constexpr int HD = 128;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kIssuerWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kIssuerWarp = 9;
 constexpr int NK = 2;
 constexpr int NV = 2;
 constexpr int kRegion = BM * 128;
 constexpr int kTileBytes = 2 * kRegion;
-constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 3;  // q, drain, K/V rings, s/p/pv
+constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 3 * 2;  // q, drain, K/V rings, s/p/pv per unit
 constexpr int kOffMisc = 8 * kNumBars;
 constexpr int kSmallBytes = kOffMisc + 16;
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffQ = 0;                         // Q_0, Q_1
+constexpr int kOffK = kOffQ + 2 * kTileBytes;
 constexpr int kOffV = kOffK + NK * kTileBytes;
 constexpr int kDataBytes = kOffV + NV * kTileBytes;
 constexpr int kSmemBytes = kSmallBytes + 1023 + kDataBytes;
@@ -49,8 +54,8 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0, "swizzled operands need 1024-byte alignment");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kTmemCols = 256;  // S/P 0-127, O 128-255
-constexpr uint32_t kTmemO = 128;
+constexpr uint32_t kTmemCols = 512;  // S_0/P_0 0-127, S_1/P_1 128-255, O_0 256-383, O_1 384-511
+constexpr uint32_t kTmemO = 256;
 
 struct PrefixParams {
   __nv_bfloat16* out;          // [B, Hq, D]
@@ -101,8 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int G = p.group;
-  const int spt = BM / G;                        // sequences per CTA
-  const int s0 = blockIdx.x * spt;               // first sequence of the CTA
+  const int spt = BM / G;                        // sequences per unit
+  const int s0 = blockIdx.x * 2 * spt;           // first sequence of the CTA (unit 0)
+  const bool two = s0 + spt < p.num_seqs;        // unit 1 has rows of real sequences
   const int g = blockIdx.y;
   const int ntiles = p.shared_len / BN;
   const int bs = 1 << p.bs_log2;
@@ -114,9 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
   uint64_t* k_empty = k_full + NK;
   uint64_t* v_full = k_empty + NK;
   uint64_t* v_empty = v_full + NV;
-  uint64_t* s_full = v_empty + NV;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* pv_done = p_full + 1;
+  uint64_t* s_full = v_empty + NV;   // [2 units] each
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(small + kOffMisc + 8);
 
@@ -131,9 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&s_full[u], 1);
+      mbar_init(&p_full[u], 4);
+      mbar_init(&pv_done[u], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     // every sequence of the CTA must hold the shared blocks at the prefix positions
     // it uses (the caller's statement of what is shared); a difference is reported
     const int nsb = p.shared_len >> p.bs_log2;
-    for (int i = lane; i < spt * nsb; i += 32) {
+    for (int i = lane; i < 2 * spt * nsb; i += 32) {
       const int s = s0 + i / nsb, b = i % nsb;
       if (s >= p.num_seqs || (b << p.bs_log2) >= __ldg(p.context_lens + s)) continue;
       const int id = __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b);
@@ -184,9 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
       // Q: G heads x 128/G sequences per box, rows in (sequence, head) order
-      mbar_arrive_expect_tx(bar_q, kTileBytes);
-      tma_load_3d(smem + kOffQ, &tmQ, bar_q, 0, g * G, s0);
-      tma_load_3d(smem + kOffQ + kRegion, &tmQ, bar_q, 64, g * G, s0);
+      mbar_arrive_expect_tx(bar_q, (two ? 2 : 1) * kTileBytes);
+      for (int u = 0; u < (two ? 2 : 1); ++u) {
+        tma_load_3d(smem + kOffQ + u * kTileBytes, &tmQ, bar_q, 0, g * G, s0 + u * spt);
+        tma_load_3d(smem + kOffQ + u * kTileBytes + kRegion, &tmQ, bar_q, 64, g * G, s0 + u * spt);
+      }
     }
     int k_issued = 0, v_issued = 0;
     for (int j = 0; j < ntiles; ++j) {
@@ -211,53 +221,58 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);
-      const uint32_t sQ = smem_u32(smem + kOffQ);
-      auto score = [&](int j) -> bool {
+      const int nu = two ? 2 : 1;
+      auto score = [&](int u, int j) -> bool {
         const int ks = j % NK;
         if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t sK = smem_u32(smem + kOffK + ks * kTileBytes);
+        const uint64_t aQ = smem_desc_sw128(smem_u32(smem + kOffQ + u * kTileBytes), 16, 1024);
+        const uint64_t bK = smem_desc_sw128(smem_u32(smem + kOffK + ks * kTileBytes), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-          tc_mma_f16_ss(tmem, smem_desc_sw128(sQ + off, 16, 1024),
-                        smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          tc_mma_f16_ss(tmem + u * 128, desc_advance(aQ, off), desc_advance(bK, off), idS,
+                        kk > 0 ? 1u : 0u);
         }
-        tc_commit(s_full);
-        tc_commit(&k_empty[ks]);
+        tc_commit(&s_full[u]);
+        if (u == nu - 1) tc_commit(&k_empty[ks]);  // K(j) frees after its last reader
         return true;
       };
-      auto pv = [&](int t) -> bool {
+      auto pv = [&](int u, int t) -> bool {
         const int vs = t % NV;
-        if (!wait_or_abort(p_full, t & 1, p.err, abort_flag, p.wait_ns) ||
+        if (!wait_or_abort(&p_full[u], t & 1, p.err, abort_flag, p.wait_ns) ||
             !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, p.wait_ns))
           return false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + kOffV + vs * kTileBytes);
+        const uint64_t bV = smem_desc_sw128(smem_u32(smem + kOffV + vs * kTileBytes), kRegion, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(sV + kk * 16 * 128, kRegion, 1024);
-          tc_mma_f16_ts(tmem + kTmemO, tmem + kk * 8, bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(pv_done);
-        tc_commit(&v_empty[vs]);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          tc_mma_f16_ts(tmem + kTmemO + u * 128, tmem + u * 128 + kk * 8,
+                        desc_advance(bV, kk * 16 * 128), idO, (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&pv_done[u]);
+        if (u == nu - 1) tc_commit(&v_empty[vs]);
         return true;
       };
-      bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns) && score(0);
+      bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
+      for (int u = 0; ok && u < nu; ++u) ok = score(u, 0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        ok = pv(j);
-        if (ok && j + 1 < ntiles) ok = score(j + 1);
+        for (int u = 0; ok && u < nu; ++u) {
+          ok = pv(u, j);
+          if (ok && j + 1 < ntiles) ok = score(u, j + 1);
+        }
       }
       tc_commit(mma_drain);
       mbar_wait(mma_drain, 0, p.err);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax + output
-    const int r = tid;                                  // query row == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off;
-    const uint32_t tO = tmem + kTmemO + lane_off;
-    const int s = s0 + r / G;
+    const int u = warp >> 2;
+    if (u == 0 || two) {
+    const int r = tid & 127;                            // query row == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + u * 128 + lane_off;
+    const uint32_t tO = tmem + kTmemO + u * 128 + lane_off;
+    const int s = s0 + u * spt + r / G;
     const int h = g * G + r % G;
     int ctx = s < p.num_seqs ? __ldg(p.context_lens + s) : 0;
     if (ctx > p.max_context_len) {
@@ -268,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     float m = -INFINITY, l = 0.f;
     bool failed = false;
     for (int j = 0; j < ntiles; ++j) {
-      failed |= !wait_or_abort(s_full, j & 1, p.err, abort_flag, p.wait_ns);
+      failed |= !wait_or_abort(&s_full[u], j & 1, p.err, abort_flag, p.wait_ns);
       tc_fence_after();
       float sv[BN];
 #pragma unroll
@@ -324,9 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[u]);
     }
-    failed |= !wait_or_abort(pv_done, (ntiles - 1) & 1, p.err, abort_flag, p.wait_ns);
+    failed |= !wait_or_abort(&pv_done[u], (ntiles - 1) & 1, p.err, abort_flag, p.wait_ns);
     tc_fence_after();
     const bool mine = s < p.num_seqs && !failed;
     const bool whole = ctx <= p.shared_len;          // the context ends inside the prefix
@@ -359,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     if (mine && !whole) {
       p.ws_ml[row * p.max_parts * 2 + 0] = m;
       p.ws_ml[row * p.max_parts * 2 + 1] = l;
+    }
     }
   }
 
@@ -405,8 +421,8 @@ cudaError_t launch_shared_prefix(const DecodeLaunch& a, const int32_t* shared_bl
   cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(shared_prefix_kernel),
                                           kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int spt = BM / G;
-  dim3 grid((a.num_seqs + spt - 1) / spt, a.cache.num_kv_heads);
+  const int spt = BM / G;  // sequences per 128-row unit; two units per CTA
+  dim3 grid((a.num_seqs + 2 * spt - 1) / (2 * spt), a.cache.num_kv_heads);
   shared_prefix_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
