@@ -48,12 +48,17 @@
 //     l keeps summing 2^(x_j - m) in fp32, and the output is O^T 2^(R - m) / l;
 //   * q (bf16) becomes three e4m3 terms with one fp32 scale per head, hi = e4m3(q/s),
 //     mid = e4m3(q/s - hi), lo = e4m3(q/s - hi - mid), written by the scheduler warp;
-//     S^T accumulates K hi^T + K mid^T + K lo^T (about 2^-13 relative error on a typical
-//     q element: a score error is multiplied by the score's size in the exponent, so
-//     peaked softmaxes need q this exact; K's codes are exact);
-//   * P' becomes hi = e4m3(P') and lo = e4m3(128 (P' - hi)), accumulated into two
-//     O^T accumulators combined as O_hi + O_lo / 128 (about 2^-8 relative on P', and
-//     an absolute floor near 2^-17, so small probabilities keep their precision).
+//     the three terms are the 48 rows of one B operand, so one product gives
+//     [K hi^T | K mid^T | K lo^T] and the softmax adds the three column groups (about
+//     2^-13 relative error on a typical q element: a score error is multiplied by the
+//     score's size in the exponent, so peaked softmaxes need q this exact; K's codes
+//     are exact);
+//   * P' becomes hi = e4m3(P') and lo = e4m3(128 (P' - hi)), the 32 rows of one B
+//     operand, so one product fills two side-by-side O^T accumulators combined as
+//     O_hi + O_lo / 128 (about 2^-8 relative on P', and an absolute floor near 2^-17,
+//     so small probabilities keep their precision).
+// Per tile that is 4 + 4 MMA instructions (K = 32 bytes each): the single issuing
+// thread, not the tensor core, sets the pace of small products like these.
 // Before a CTA ends, its producer waits for every copy it started and its issuer for
 // every MMA it issued (with the full time limit, even when the roles gave up early),
 // so no asynchronous write outlives the CTA's shared and tensor memory.
@@ -127,10 +132,14 @@ struct Cfg {
   // e4m3: the K-scale ring [NSC] and each V slot's scales [NV], 1 KB each
   static constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
   static constexpr int kSmemBytes = (F8 ? kOffScl + (NSC + NV) * kSclBytes : kOffMisc + 64) + 1024;
-  // TMEM columns: S^T[NS] at 16 i; O^T[NO] at 64 + 16 i; e4m3 low-term O^T at 112 + 16 i
-  static constexpr uint32_t kTmemO = 64;
-  static constexpr uint32_t kTmemOlo = 64 + 16 * NO;
-  static constexpr uint32_t kTmemCols = F8 ? 256 : 128;
+  // TMEM columns. bf16: S^T[NS] 16 columns each, then O^T[NO] 16 each. e4m3: S^T[NS] 48
+  // columns each (the hi, mid and lo q terms' products side by side: one MMA with the
+  // three terms stacked as N = 48), then O^T[NO] 32 each (P's hi and lo terms stacked as
+  // N = 32: the hi accumulator, then the lo one)
+  static constexpr uint32_t kSCols = F8 ? NQ * kQTerms : NQ;
+  static constexpr uint32_t kOCols = F8 ? 2 * NQ : NQ;
+  static constexpr uint32_t kTmemO = NS * kSCols;
+  static constexpr uint32_t kTmemCols = F8 ? 512 : 128;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffQ % 1024 == 0 && kOffP % 1024 == 0,
                 "128-byte-swizzled TMA / MMA operands need 1024-byte alignment");
@@ -138,8 +147,7 @@ struct Cfg {
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kOffSched % 16 == 0 && kOffDesc % 16 == 0 && kOffEpi % 16 == 0 && kEpiBytes % 16 == 0,
                 "descriptor slots");
-  static_assert(kTmemOlo + (F8 ? 16 * NO : 0) <= kTmemCols && kTmemO + 16 * NO <= kTmemCols,
-                "tensor memory columns");
+  static_assert(kTmemO + kOCols * NO <= kTmemCols, "tensor memory columns");
 };
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -237,22 +245,6 @@ __device__ __forceinline__ unsigned tagged_arrive(unsigned long long* ctr, unsig
 }
 
 // bounded wait that also gives up once another role has given up
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
-                                              volatile int* abort_flag,
-                                              unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      flag_error(err, PA_DEV_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -730,42 +722,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     }
   } else if (warp == 5) {
     // ======================================================== tensor-core issuer
-    if (lane == 0) {
-      // bf16: K K-major, Q^T K-major; V^T MN-major, P^T K-major (same for e4m3)
-      constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TM, NQ, 0, 0) : idesc_bf16_f32(TM, NQ, 0, 0);
-      constexpr uint32_t idO = F8 ? idesc_e4m3_f32(HD, NQ, 1, 0) : idesc_bf16_f32(HD, NQ, 1, 0);
+    // the whole warp runs this loop (its descriptors stay warp-uniform); one elected lane
+    // issues each MMA and commit
+    {
+      // bf16: K K-major, Q^T K-major; V^T MN-major, P^T K-major (same for e4m3, with the
+      // q terms stacked as N = 48 and P's two terms as N = 32)
+      constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TM, NQ * kQTerms, 0, 0) : idesc_bf16_f32(TM, NQ, 0, 0);
+      constexpr uint32_t idO = F8 ? idesc_e4m3_f32(HD, 2 * NQ, 1, 0) : idesc_bf16_f32(HD, NQ, 1, 0);
       const uint32_t sP = smem_u32(smem + C::kOffP);
       unsigned j = 0;  // tiles whose score MMA was issued
       // O^T(obuf) += V^T(t) P^T(t); `first` overwrites instead of accumulating
       auto pv = [&](unsigned t, bool first, int obuf, int item) -> bool {
         const int b = t % NP;
         const int vs = t % NV;
-        if (!wait_or_abort(&p_full[b], (t / NP) & 1, p.err, abort_flag, wl) ||
-            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, wl))
+        if (!warp_wait_or_abort(&p_full[b], (t / NP) & 1, p.err, abort_flag, wl) ||
+            !warp_wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, wl))
           return false;
         // the first value MMA of an item overwrites O(obuf): the epilogue of the item
         // that used this accumulator NO items ago must have read it
         if (first && item >= NO &&
-            !wait_or_abort(&o_free[obuf], ((item / NO) - 1) & 1, p.err, abort_flag, wl))
+            !warp_wait_or_abort(&o_free[obuf], ((item / NO) - 1) & 1, p.err, abort_flag, wl))
           return false;
         tc_fence_after();
         // one descriptor per operand, stepped by constant offsets (see desc_advance)
         const uint64_t aV = smem_desc_sw128(smem_u32(smem + C::kOffV + vs * kTileBytes),
                                             kRegion, 1024);
         const uint64_t bP = smem_desc_sw128(sP + b * kPBytes, 16, 1024);
-        const uint32_t dO = tmem + C::kTmemO + obuf * 16;
+        const uint32_t dO = tmem + C::kTmemO + obuf * C::kOCols;
         if (F8) {
-          // 32 positions (4 rows of 8-row swizzle atoms) per instruction; the hi term of
-          // P' into O, the lo term into the second accumulator
-          const uint32_t dOlo = tmem + C::kTmemOlo + obuf * 16;
+          // 32 positions (4 rows of 8-row swizzle atoms) per instruction; P's hi and lo
+          // terms are one B operand of 32 rows, so O_hi and O_lo come out side by side
 #pragma unroll
           for (int kk = 0; kk < TM / 32; ++kk)
             tc_mma_f8_ss(dO, desc_advance(aV, kk * 32 * 128), desc_advance(bP, kk * 32), idO,
                          (first && kk == 0) ? 0u : 1u);
-#pragma unroll
-          for (int kk = 0; kk < TM / 32; ++kk)
-            tc_mma_f8_ss(dOlo, desc_advance(aV, kk * 32 * 128),
-                         desc_advance(bP, kQRegion + kk * 32), idO, (first && kk == 0) ? 0u : 1u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < TM / 16; ++kk)
@@ -781,18 +771,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       bool ok = true;
       while (ok) {
         const int slot = k % QN;
-        if (!wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
+        if (!warp_wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const ItemDesc d = descs[slot];
         if (d.stop) break;
         // e4m3: the scheduler writes the item's q terms after publishing the item
-        if (F8 && !wait_or_abort(&q_ready[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
+        if (F8 && !warp_wait_or_abort(&q_ready[slot], (k / QN) & 1, p.err, abort_flag, wl)) break;
         const uint32_t sQ = smem_u32(smem + C::kOffQ + slot * C::kQBytes);
         const int obuf = k % NO;
         for (int i = 0; i < d.ntiles; ++i, ++j) {
           const int ks = j % NK;
           const int sb = j % NS;
-          if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, wl) ||
-              (j >= NS && !wait_or_abort(&s_free[sb], ((j / NS) - 1) & 1, p.err, abort_flag, wl))) {
+          if (!warp_wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, wl) ||
+              (j >= NS && !warp_wait_or_abort(&s_free[sb], ((j / NS) - 1) & 1, p.err, abort_flag, wl))) {
             ok = false;
             break;
           }
@@ -800,17 +790,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           const uint64_t aK = smem_desc_sw128(smem_u32(smem + C::kOffK + ks * kTileBytes), 16, 1024);
           const uint64_t bQ = smem_desc_sw128(sQ, 16, 1024);
           if (F8) {
-            // S^T = K hi^T + K mid^T + K lo^T: 32 head dims (bytes) of each row per
-            // instruction
+            // [K hi^T | K mid^T | K lo^T] in one product: the three q terms are the 48 rows
+            // of one B operand; 32 head dims (bytes) of each row per instruction
 #pragma unroll
-            for (int kk = 0; kk < kQTerms * (HD / 32); ++kk)
-              tc_mma_f8_ss(tmem + sb * 16, desc_advance(aK, (kk & 3) * 32),
-                           desc_advance(bQ, (kk >> 2) * kQRegion + (kk & 3) * 32), idS,
-                           kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < HD / 32; ++kk)
+              tc_mma_f8_ss(tmem + sb * C::kSCols, desc_advance(aK, kk * 32),
+                           desc_advance(bQ, kk * 32), idS, kk > 0 ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-              tc_mma_f16_ss(tmem + sb * 16, desc_advance(aK, (kk >> 2) * kRegion + (kk & 3) * 32),
+              tc_mma_f16_ss(tmem + sb * C::kSCols, desc_advance(aK, (kk >> 2) * kRegion + (kk & 3) * 32),
                             desc_advance(bQ, (kk >> 2) * kQRegion + (kk & 3) * 32), idS,
                             kk > 0 ? 1u : 0u);
           }
@@ -881,7 +870,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         failed |= !wait_or_abort(&s_full[sb], (j / NS) & 1, p.err, abort_flag, wl);
         tc_fence_after();
         float sv[16];
-        tmem_ld16(tmem + sb * 16 + lane_off, sv);
+        tmem_ld16(tmem + sb * C::kSCols + lane_off, sv);
+        if constexpr (F8) {
+          // S = products with the hi, mid and lo q terms, summed
+          float s1[16], s2[16];
+          tmem_ld16(tmem + sb * C::kSCols + NQ + lane_off, s1);
+          tmem_ld16(tmem + sb * C::kSCols + 2 * NQ + lane_off, s2);
+          tc_wait_ld();
+#pragma unroll
+          for (int h = 0; h < G; ++h) sv[h] = (sv[h] + s1[h]) + s2[h];
+        }
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -1021,17 +1019,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           failed |= !wait_or_abort(&pv_done[t % NP], (t / NP) & 1, p.err, abort_flag, wl);
           tc_fence_after();
           float o[16];
-          tmem_ld16(tmem + C::kTmemO + obuf * 16 + lane_off, o);
+          tmem_ld16(tmem + C::kTmemO + obuf * C::kOCols + lane_off, o);
           tc_wait_ld();
 #pragma unroll
           for (int h = 0; h < G; ++h) o[h] *= alpha[h];
-          tmem_st16(tmem + C::kTmemO + obuf * 16 + lane_off, o);
-          if (F8) {
-            tmem_ld16(tmem + C::kTmemOlo + obuf * 16 + lane_off, o);
+          tmem_st16(tmem + C::kTmemO + obuf * C::kOCols + lane_off, o);
+          if (F8) {  // the lo accumulator, next to the hi one
+            tmem_ld16(tmem + C::kTmemO + obuf * C::kOCols + NQ + lane_off, o);
             tc_wait_ld();
 #pragma unroll
             for (int h = 0; h < G; ++h) o[h] *= alpha[h];
-            tmem_st16(tmem + C::kTmemOlo + obuf * 16 + lane_off, o);
+            tmem_st16(tmem + C::kTmemO + obuf * C::kOCols + NQ + lane_off, o);
           }
           tc_wait_st();
         }
@@ -1098,10 +1096,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       failed |= !wait_or_abort(&o_full[b], (k / NO) & 1, p.err, abort_flag, wl);
       tc_fence_after();
       float o[16];
-      tmem_ld16(tmem + C::kTmemO + b * 16 + lane_off, o);
+      tmem_ld16(tmem + C::kTmemO + b * C::kOCols + lane_off, o);
       if (F8) {
         float olo[16];
-        tmem_ld16(tmem + C::kTmemOlo + b * 16 + lane_off, olo);
+        tmem_ld16(tmem + C::kTmemO + b * C::kOCols + NQ + lane_off, olo);
         tc_wait_ld();
 #pragma unroll
         for (int h = 0; h < G; ++h) o[h] = fmaf(olo[h], 1.f / kPLoScale, o[h]) * fac[h];

@@ -99,23 +99,6 @@ struct PrefillParams {
   uint4* v_rows;
 };
 
-// bounded wait that also gives up when another role has already given up
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
-                                              volatile int* abort_flag,
-                                              unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      flag_error(err, PA_DEV_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
 // One unit's place in the batch: its query tile, head, visible range and tile count.
 struct Unit {
   int qt, h, rows_valid, pos_max, ntiles;
@@ -329,14 +312,16 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
     }
   } else if (warp == kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop (its descriptors stay warp-uniform); one elected lane
+    // issues each MMA and commit
+    {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);  // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);  // P (TMEM), V MN-major
       // S_u(j) over S_u's columns once K(j) has landed (S_u(j-1) was read and P_u(j-1)
       // consumed by the value MMA queued before it); K(j) frees after its last reader
       auto score = [&](int u, int j) -> bool {
         const int ks = j % NK;
-        if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns))
+        if (!warp_wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns))
           return false;
         tc_fence_after();
         // one descriptor per operand, stepped by constant offsets (see desc_advance)
@@ -355,8 +340,8 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
       // O_u += P_u(t) V(t), once the softmax has written P_u(t) and V(t) has landed
       auto pv = [&](int u, int t) -> bool {
         const int vs = t % NV;
-        if (!wait_or_abort(&p_full[u], t & 1, p.err, abort_flag, p.wait_ns) ||
-            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, p.wait_ns))
+        if (!warp_wait_or_abort(&p_full[u], t & 1, p.err, abort_flag, p.wait_ns) ||
+            !warp_wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, p.wait_ns))
           return false;
         tc_fence_after();
         const uint32_t tP = tmem + u * 128;
@@ -369,7 +354,7 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
         if (u == 1 || t >= nt1) tc_commit(&v_empty[vs]);
         return true;
       };
-      bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
+      bool ok = warp_wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
       if (ok) ok = score(0, 0);
       if (ok && nt1 > 0) ok = score(1, 0);
       for (int j = 0; ok && j < nmax; ++j) {

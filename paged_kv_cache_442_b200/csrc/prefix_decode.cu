@@ -78,22 +78,6 @@ struct PrefixParams {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
-                                              volatile int* abort_flag,
-                                              unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      flag_error(err, PA_DEV_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
 __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const PrefixParams p) {
@@ -218,13 +202,15 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     }
   } else if (warp == kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop (its descriptors stay warp-uniform); one elected lane
+    // issues each MMA and commit
+    {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, HD, 0, 1);
       const int nu = two ? 2 : 1;
       auto score = [&](int u, int j) -> bool {
         const int ks = j % NK;
-        if (!wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns)) return false;
+        if (!warp_wait_or_abort(&k_full[ks], (j / NK) & 1, p.err, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         const uint64_t aQ = smem_desc_sw128(smem_u32(smem + kOffQ + u * kTileBytes), 16, 1024);
         const uint64_t bK = smem_desc_sw128(smem_u32(smem + kOffK + ks * kTileBytes), 16, 1024);
@@ -240,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       };
       auto pv = [&](int u, int t) -> bool {
         const int vs = t % NV;
-        if (!wait_or_abort(&p_full[u], t & 1, p.err, abort_flag, p.wait_ns) ||
-            !wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, p.wait_ns))
+        if (!warp_wait_or_abort(&p_full[u], t & 1, p.err, abort_flag, p.wait_ns) ||
+            !warp_wait_or_abort(&v_full[vs], (t / NV) & 1, p.err, abort_flag, p.wait_ns))
           return false;
         tc_fence_after();
         const uint64_t bV = smem_desc_sw128(smem_u32(smem + kOffV + vs * kTileBytes), kRegion, 1024);
@@ -253,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
         if (u == nu - 1) tc_commit(&v_empty[vs]);
         return true;
       };
-      bool ok = wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
+      bool ok = warp_wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
       for (int u = 0; ok && u < nu; ++u) ok = score(u, 0);
       for (int j = 0; ok && j < ntiles; ++j) {
         for (int u = 0; ok && u < nu; ++u) {
