@@ -714,12 +714,20 @@ def main():
 
     step_ms = max_over_ranks(total_ms / args.steps, pg, torch, "cuda")
     bytes_step = (decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)) + store_bytes(w)
+    unique = None
+    if shared:
+        # the shared prefix is read once for all sequences: the bytes the step must move
+        # are the unique ones (every distinct K/V row once, q, out)
+        unique = w.kv_bytes_unique() + 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+        bytes_step = unique + store_bytes(w)
     job_bytes = sum_over_ranks(bytes_step, pg, torch, "cuda")
     value = job_gbps(job_bytes, step_ms)
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     attn_bytes = decode_bytes(w) if w.kind == "decode" else prefill_bytes(w)
     if runner.fused:
         attn_bytes += store_bytes(w)  # the new rows are read and written by the same launch
+    if unique is not None:
+        attn_bytes = unique
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     if w.kind == "decode":
         kname = ("pa_store_decode (persistent tcgen05 decode; new-row store and split-K merge inside)"
@@ -773,7 +781,9 @@ def main():
                    "context_lens": f"{cfg.ctx_dist}[{cfg.ctx_lo},{cfg.ctx_hi}] sum={int(w.context_lens.sum())}",
                    "partition_size": getattr(runner, "P", None),
                    "parallelism": f"replicas x{world} (independent batches)",
-                   "l2": "flushed before every step by reading a 256 MiB buffer (clean lines; outside the step events)"},
+                   "l2": "flushed before every step by reading a 256 MiB buffer (clean lines; outside the step events)",
+                   "bytes": ("unique: every distinct K/V row once (the shared prefix is attended once), q, out"
+                             if shared else "every sequence's K/V rows, q, out (+ the new rows when stored)")},
         "steps_per_s": round(1e3 / step_ms * world, 1),
         "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
         "pct_of_datasheet_8tbs": round(100 * value / world / DATASHEET_HBM_GBS, 1),

@@ -16,14 +16,15 @@
 // decode kernel's partitions), which the persistent decode over the remaining
 // positions merges in.
 // Each CTA takes two such tiles of 128 query rows (units 0 and 1, consecutive rows of
-// one kv head) that read the same shared tiles, and the tensor core alternates between
-// them: issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so one unit's softmax runs
+// one kv head) that read the same shared tiles (one tile when two per CTA would leave
+// SMs idle), and the tensor core alternates between them: issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so one unit's softmax runs
 // while the other unit's products execute (P_u is written over S_u in TMEM, and
 // S_u(j+1) done implies PV_u(j) done).
 // Roles (320 threads): warps 0-3 / 4-7 softmax + output of unit 0 / 1, warp 8 TMA
 // producer (both Q tiles, then K and V of the shared blocks in two-deep rings),
 // warp 9 TMEM owner (all 512 columns: S_0/P_0, S_1/P_1, O_0, O_1) and MMA issuer. The
-// producer warp also checks every sequence of the CTA's rows against the shared blocks.
+// softmax warps first check every sequence of the CTA's rows against the shared blocks
+// (while the first tiles load).
 #include <cuda_bf16.h>
 
 #include "pa_internal.h"
@@ -72,6 +73,7 @@ struct PrefixParams {
   int num_blocks;
   int bs_log2;
   int shared_len;              // multiple of 128
+  int units;                   // 128-row units per CTA: 2, or 1 when two would leave SMs idle
   int max_parts;
   int max_context_len;
   float scale_log2;
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
   const int lane = tid & 31;
   const int G = p.group;
   const int spt = BM / G;                        // sequences per unit
-  const int s0 = blockIdx.x * 2 * spt;           // first sequence of the CTA (unit 0)
-  const bool two = s0 + spt < p.num_seqs;        // unit 1 has rows of real sequences
+  const int s0 = blockIdx.x * p.units * spt;     // first sequence of the CTA (unit 0)
+  const bool two = p.units == 2 && s0 + spt < p.num_seqs;  // unit 1 has rows of real sequences
   const int g = blockIdx.y;
   const int ntiles = p.shared_len / BN;
   const int bs = 1 << p.bs_log2;
@@ -145,15 +147,6 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       if (lane == 0) okw = wait_or_abort(bar, parity, p.err, abort_flag, p.wait_ns) ? 1 : 0;
       return __shfl_sync(0xffffffffu, okw, 0) != 0;
     };
-    // every sequence of the CTA must hold the shared blocks at the prefix positions
-    // it uses (the caller's statement of what is shared); a difference is reported
-    const int nsb = p.shared_len >> p.bs_log2;
-    for (int i = lane; i < 2 * spt * nsb; i += 32) {
-      const int s = s0 + i / nsb, b = i % nsb;
-      if (s >= p.num_seqs || (b << p.bs_log2) >= __ldg(p.context_lens + s)) continue;
-      const int id = __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b);
-      if (id != __ldg(p.shared_blocks + b)) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
-    }
     const int rows = bs < BN ? bs : BN;
     const int nbox = BN / rows;
     const uint64_t keep = policy_evict_last();  // the prefix is read by every CTA of g
@@ -252,6 +245,19 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax + output
+    // First, while the first tiles load: every sequence of the CTA must hold the shared
+    // blocks at the prefix positions it uses (the caller's statement of what is
+    // shared); a difference is reported. (256 threads: these dependent global reads
+    // would hold up the producer's first loads by tens of microseconds.)
+    {
+      const int nsb = p.shared_len >> p.bs_log2;
+      for (int i = tid; i < p.units * spt * nsb; i += 8 * 32) {
+        const int s = s0 + i / nsb, b = i % nsb;
+        if (s >= p.num_seqs || (b << p.bs_log2) >= __ldg(p.context_lens + s)) continue;
+        const int id = __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b);
+        if (id != __ldg(p.shared_blocks + b)) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+      }
+    }
     const int u = warp >> 2;
     if (u == 0 || two) {
     const int r = tid & 127;                            // query row == TMEM lane
@@ -407,8 +413,12 @@ cudaError_t launch_shared_prefix(const DecodeLaunch& a, const int32_t* shared_bl
   cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(shared_prefix_kernel),
                                           kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int spt = BM / G;  // sequences per 128-row unit; two units per CTA
-  dim3 grid((a.num_seqs + 2 * spt - 1) / (2 * spt), a.cache.num_kv_heads);
+  // sequences per 128-row unit; two units per CTA (one unit's softmax overlaps the
+  // other's products) unless that leaves SMs idle, then one (more SMs beat the overlap)
+  const int spt = BM / G;
+  const int tiles = (a.num_seqs + spt - 1) / spt;
+  p.units = ((tiles + 1) / 2) * a.cache.num_kv_heads < sm_count() ? 1 : 2;
+  dim3 grid((a.num_seqs + p.units * spt - 1) / (p.units * spt), a.cache.num_kv_heads);
   shared_prefix_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
