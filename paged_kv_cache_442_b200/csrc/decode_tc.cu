@@ -90,7 +90,6 @@ constexpr int QN = 2;          // item queue depth (producer -> issuer, softmax)
 constexpr int QS = 2;          // scheduler queue depth: one item prepared ahead (deeper
                                // queues reserve work early and unbalance the tail)
 constexpr int NO = 3;          // O^T accumulators in TMEM (one per item in flight)
-constexpr int kPass = 1;       // tiles per softmax pass (one max exchange per pass)
 constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-9, scheduler 10
 constexpr float kRescaleLog2 = 8.f;  // rescale when the max grows by more than this
 constexpr int kQRegion = NQ * 128;           // 16 rows x 128 bytes (2 KB)
@@ -766,12 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TM, NQ * kQTerms, 0, 0) : idesc_bf16_f32(TM, NQ, 0, 0);
       constexpr uint32_t idO = F8 ? idesc_e4m3_f32(HD, 2 * NQ, 1, 0) : idesc_bf16_f32(HD, NQ, 1, 0);
       const uint32_t sP = smem_u32(smem + C::kOffP);
-      // Two cursors over the CTA's tiles. The score cursor (item ks, tile is, CTA tile js)
-      // runs ahead of the value cursor (item kp, tile ip, CTA tile jp): before the value
-      // MMA of tile jp it must have issued the score MMAs of the softmax pass holding jp
-      // (blocking waits), and it issues up to kLookahead - 1 more whose K tile, S buffer
-      // and item are already there (non-blocking tests), so the softmax never waits for
-      // a score product that could have run during its previous pass.
+      // Two cursors over the CTA's tiles: the score cursor (item ks, tile is, CTA tile
+      // js) runs up to kLookahead tiles ahead of the value cursor (item kp, tile ip, CTA
+      // tile jp). Both advance only on non-blocking tests of their barriers.
       constexpr unsigned kLookahead = NS;
       int ks = 0, is = 0, s_nt = 0;
       unsigned js = 0;
@@ -780,26 +776,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       int nt_ring[8];  // tile counts of the items between the two cursors
       int kp = 0, ip = 0;
       unsigned jp = 0;
-      bool ok = true;
-      // the score cursor enters its next item (false: not published yet, or a failed wait)
-      auto s_enter = [&](bool block) -> bool {
+      // the score cursor enters its next item (false: not published yet, or the stop item)
+      auto s_enter = [&]() -> bool {
         const int slot = ks % QN;
         const unsigned ph = (ks / QN) & 1;
-        if (block) {
-          if (!warp_wait_or_abort(&item_full[slot], ph, p.err, abort_flag, wl)) { ok = false; return false; }
-        } else if (!__all_sync(0xffffffffu, mbar_test_wait(&item_full[slot], ph))) {
-          return false;
-        }
+        if (!__all_sync(0xffffffffu, mbar_test_wait(&item_full[slot], ph))) return false;
         const ItemDesc d = descs[slot];
         if (d.stop) { s_end = true; return false; }
         // e4m3: the scheduler writes the item's q terms after publishing the item
-        if (F8) {
-          if (block) {
-            if (!warp_wait_or_abort(&q_ready[slot], ph, p.err, abort_flag, wl)) { ok = false; return false; }
-          } else if (!__all_sync(0xffffffffu, mbar_test_wait(&q_ready[slot], ph))) {
-            return false;
-          }
-        }
+        if (F8 && !__all_sync(0xffffffffu, mbar_test_wait(&q_ready[slot], ph))) return false;
         s_nt = d.ntiles;
         nt_ring[ks & 7] = s_nt;
         sQ = smem_u32(smem + C::kOffQ + slot * C::kQBytes);
@@ -807,21 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         s_in = true;
         return true;
       };
-      // S^T(js) (false: its K tile or S buffer is not ready, or a failed wait)
-      auto score = [&](bool block) -> bool {
-        if (!s_in && (s_end || !s_enter(block))) return false;
+      // S^T(js) (false: its item, K tile or S buffer is not ready)
+      auto score = [&]() -> bool {
+        if (!s_in && (s_end || !s_enter())) return false;
         const int kslot = js % NK;
         const int sb = js % NS;
-        if (block) {
-          if (!warp_wait_or_abort(&k_full[kslot], (js / NK) & 1, p.err, abort_flag, wl) ||
-              (js >= NS && !warp_wait_or_abort(&s_free[sb], ((js / NS) - 1) & 1, p.err, abort_flag, wl))) {
-            ok = false;
-            return false;
-          }
-        } else if (!__all_sync(0xffffffffu, mbar_test_wait(&k_full[kslot], (js / NK) & 1) &&
-                                                (js < NS || mbar_test_wait(&s_free[sb], ((js / NS) - 1) & 1)))) {
+        if (!__all_sync(0xffffffffu, mbar_test_wait(&k_full[kslot], (js / NK) & 1) &&
+                                         (js < NS || mbar_test_wait(&s_free[sb], ((js / NS) - 1) & 1))))
           return false;
-        }
         tc_fence_after();
         const uint64_t aK = smem_desc_sw128(smem_u32(smem + C::kOffK + kslot * kTileBytes), 16, 1024);
         const uint64_t bQ = smem_desc_sw128(sQ, 16, 1024);
@@ -890,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       // ahead whenever its item, K tile and S buffer are ready; when nothing is, wait
       // briefly on the barrier most likely to complete next. The idle time is bounded.
       unsigned long long idle_since = 0;
-      while (ok) {
+      while (true) {
         bool progressed = false;
         if (jp < js && pv(jp, ip == 0, kp % NO, kp)) {
           ++jp;
@@ -900,10 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             ++kp;
           }
           progressed = true;
-        } else if (js < jp + kLookahead && ks - kp < 7 && score(false)) {
+        } else if (js < jp + kLookahead && ks - kp < 7 && score()) {
           progressed = true;
         }
-        if (!ok) break;
         if (jp == js && s_end) break;  // every item done
         if (progressed) {
           idle_since = 0;
@@ -941,8 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // e4m3: byte offset of position r's scale within a tile's scale area
     const int soff = (r / srows) * sstride + (r % srows) * 4;
     int k = 0;
-    unsigned j = 0;     // tiles of this CTA done
-    unsigned pass = 0;  // passes (tile pairs) of this CTA: parity of the exchange buffers
+    unsigned j = 0;  // tiles of this CTA done
     while (true) {
       const int slot = k % QN;
       bool failed = !wait_or_abort(&item_full[slot], (k / QN) & 1, p.err, abort_flag, wl);
@@ -974,94 +950,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         lp[h] = 0.f;
         R[h] = -INFINITY;  // e4m3: O's reference, unset until a tile has a non-zero V scale
       }
-      // A pass takes kPass tiles of the item (the last pass may take fewer): one max
-      // exchange and one barrier serve them all and the reference max is the pass's.
-      // Two tiles per pass measured slower than one (the pass's P hand-offs come later,
-      // so the value MMAs and the V ring wait longer), so kPass is 1.
-      for (int i = 0; i < d.ntiles; i += kPass, ++pass) {
-        const int nt = i + 1 < d.ntiles ? kPass : 1;
-#pragma unroll
-        for (int t = 0; t < kPass; ++t)
-          if (t < nt)
-            failed |= !wait_or_abort(&s_full[(j + t) % NS], ((j + t) / NS) & 1, p.err, abort_flag, wl);
+      for (int i = 0; i < d.ntiles; ++i, ++j) {
+        const int sb = j % NS;
+        const bool valid = i * TM + r < d.n;
+        // e4m3: the tile's K and V row scales first: they land with the tiles, well
+        // before the score MMA is done, so their waits and reads overlap it
+        float skr = 1.f;
+        float svr = 0.f;  // e4m3: this position's V scale (0 past the partition)
+        if constexpr (F8) {
+          const int kl = j % NSC;
+          failed |= !wait_or_abort(&ksc_full[kl], (j / NSC) & 1, p.err, abort_flag, wl);
+          skr = *reinterpret_cast<const float*>(smem + C::kOffScl + kl * kSclBytes + soff);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ksc_empty[kl]);
+          const int vs = j % NV;
+          failed |= !wait_or_abort(&vsc_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
+          if (valid)
+            svr = *reinterpret_cast<const float*>(smem + C::kOffScl + (NSC + vs) * kSclBytes + soff);
+        }
+        failed |= !wait_or_abort(&s_full[sb], (j / NS) & 1, p.err, abort_flag, wl);
         tc_fence_after();
-        float sv[kPass][G], s1[kPass][G], s2[kPass][G];
+        float sv[G];
+        tmem_ld_cols<G>(tmem + sb * C::kSCols + lane_off, sv);
+        if constexpr (F8) {
+          // S = products with the hi, mid and lo q terms, summed
+          float s1[G], s2[G];
+          tmem_ld_cols<G>(tmem + sb * C::kSCols + NQ + lane_off, s1);
+          tmem_ld_cols<G>(tmem + sb * C::kSCols + 2 * NQ + lane_off, s2);
+          tc_wait_ld();
 #pragma unroll
-        for (int t = 0; t < kPass; ++t) {
-          if (t < nt) {
-            const uint32_t ts = tmem + ((j + t) % NS) * C::kSCols + lane_off;
-            tmem_ld_cols<G>(ts, sv[t]);
-            if constexpr (F8) {  // the products with the mid and lo q terms
-              tmem_ld_cols<G>(ts + NQ, s1[t]);
-              tmem_ld_cols<G>(ts + 2 * NQ, s2[t]);
-              if constexpr (G == 16) {  // sixteen heads: sum per tile (registers)
-                tc_wait_ld();
-#pragma unroll
-                for (int h = 0; h < G; ++h) sv[t][h] = (sv[t][h] + s1[t][h]) + s2[t][h];
-              }
-            }
-          }
+          for (int h = 0; h < G; ++h) sv[h] = (sv[h] + s1[h]) + s2[h];
         }
         tc_wait_ld();
-        if constexpr (F8 && G < 16) {  // S = the three products summed
-#pragma unroll
-          for (int t = 0; t < kPass; ++t)
-#pragma unroll
-            for (int h = 0; h < G; ++h) sv[t][h] = (sv[t][h] + s1[t][h]) + s2[t][h];
-        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&s_free[j % NS]);
-          if (nt == 2) mbar_arrive(&s_free[(j + 1) % NS]);
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+        float x[G];
+        if constexpr (F8) {
+          const float fr = p.scale_log2 * skr;
+#pragma unroll
+          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * (fr * qsg[h]) : -INFINITY;
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
         }
-        bool valid[kPass];
-        float x[kPass][G];
-        float svr[kPass];  // e4m3: this position's V scales (0 past the partition)
-#pragma unroll
-        for (int t = 0; t < kPass; ++t) {
-          valid[t] = t < nt && (i + t) * TM + r < d.n;
-          svr[t] = 0.f;
-          if constexpr (F8) {
-            if (t < nt) {
-              const unsigned jt = j + t;
-              const int kl = jt % NSC;
-              failed |= !wait_or_abort(&ksc_full[kl], (jt / NSC) & 1, p.err, abort_flag, wl);
-              const float skr = *reinterpret_cast<const float*>(smem + C::kOffScl + kl * kSclBytes + soff);
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&ksc_empty[kl]);
-              const int vs = jt % NV;
-              failed |= !wait_or_abort(&vsc_full[vs], (jt / NV) & 1, p.err, abort_flag, wl);
-              if (valid[t])
-                svr[t] = *reinterpret_cast<const float*>(smem + C::kOffScl + (NSC + vs) * kSclBytes + soff);
-              const float fr = p.scale_log2 * skr;
-#pragma unroll
-              for (int h = 0; h < G; ++h) x[t][h] = valid[t] ? sv[t][h] * (fr * qsg[h]) : -INFINITY;
-            } else {
-#pragma unroll
-              for (int h = 0; h < G; ++h) x[t][h] = -INFINITY;
-            }
-          } else {
-#pragma unroll
-            for (int h = 0; h < G; ++h) x[t][h] = valid[t] ? sv[t][h] * p.scale_log2 : -INFINITY;
-          }
-        }
-        // per-head max over the pair: warp shuffles, then across the 4 warps
-        float* rb = red + (pass & 1) * 4 * NQ;
+        // per-head max over the tile: warp shuffles, then across the 4 warps
+        float* rb = red + (j & 1) * 4 * NQ;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          float v = x[0][h];
-#pragma unroll
-          for (int t = 1; t < kPass; ++t) v = fmaxf(v, x[t][h]);
+          float v = x[h];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) rb[warp * NQ + h] = v;
         }
-        float* svb = red + 3 * 4 * NQ + (pass & 1) * 4;  // e4m3: the pair's largest V scale
+        float* svb = red + 3 * 4 * NQ + (j & 1) * 4;  // e4m3: the tile's largest V scale
         if (F8) {
-          float v = svr[0];
-#pragma unroll
-          for (int t = 1; t < kPass; ++t) v = fmaxf(v, svr[t]);
+          float v = svr;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) svb[warp] = v;
@@ -1069,13 +1013,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         named_bar_sync(1, 128);
         bool rescale = false;
         float alpha[G];
-        float pp[kPass][G];  // P' (e4m3) or P (bf16) of this position per head, per tile
+        float pp[G];  // e4m3: P' of this position per head
         if constexpr (F8) {
-          // bound of P' over the pair: 2^(max x + log2 max s_v - R)
+          // bound of P' over the tile: 2^(max x + log2 max s_v - R)
           const float lsm = lg2_approx(fmaxf(fmaxf(svb[0], svb[1]), fmaxf(svb[2], svb[3])));
-          float lsv[kPass];  // -inf for s_v = 0 (and past the partition)
-#pragma unroll
-          for (int t = 0; t < kPass; ++t) lsv[t] = lg2_approx(svr[t]);
+          const float lsv = lg2_approx(svr);  // -inf for s_v = 0 (and past the partition)
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
@@ -1086,9 +1028,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
               lp[h] *= ex2_approx(m[h] - mx);
               m[h] = mx;
             }
-#pragma unroll
-            for (int t = 0; t < kPass; ++t) lp[h] += valid[t] ? ex2_approx(x[t][h] - m[h]) : 0.f;
-            // O's reference: set by the first pair with a non-zero V scale (O is exactly
+            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
+            lp[h] += pr;
+            // O's reference: set by the first tile with a non-zero V scale (O is exactly
             // 0 before it), raised when the bound would pass 2^kPBoundLog2
             alpha[h] = 1.f;
             const float bnd = mx + lsm;
@@ -1100,9 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
               R[h] = rn;
               rescale = true;
             }
-#pragma unroll
-            for (int t = 0; t < kPass; ++t)
-              pp[t][h] = (valid[t] && R[h] > -INFINITY) ? ex2_approx(x[t][h] + lsv[t] - R[h]) : 0.f;
+            pp[h] = (valid && R[h] > -INFINITY) ? ex2_approx(x[h] + lsv - R[h]) : 0.f;
           }
         } else {
 #pragma unroll
@@ -1110,69 +1050,60 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
             alpha[h] = 1.f;
             if (i == 0) {
-              m[h] = mx;  // reference max of this item (every pair has a valid position)
+              m[h] = mx;  // reference max of this item (every tile has a valid position)
             } else if (mx > m[h] + kRescaleLog2) {
               alpha[h] = ex2_approx(m[h] - mx);
               m[h] = mx;
               rescale = true;
             }
-            float ps = 0.f;
-#pragma unroll
-            for (int t = 0; t < kPass; ++t) {
-              pp[t][h] = valid[t] ? ex2_approx(x[t][h] - m[h]) : 0.f;
-              ps += pp[t][h];
-            }
-            lp[h] = lp[h] * alpha[h] + ps;
+            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
+            lp[h] = lp[h] * alpha[h] + pr;
+            pp[h] = pr;
           }
         }
+        // this P^T buffer was last read by the value MMA of tile j - NP
+        const int pb = j % NP;
+        if (j >= NP)
+          failed |= !wait_or_abort(&pv_done[pb], ((j / NP) - 1) & 1, p.err, abort_flag, wl);
+        if constexpr (F8) {
+          // row h of P^T (K-major, 128 positions = 128 bytes, 128-byte swizzle): byte r
+          uint8_t* pt = smem + C::kOffP + pb * kPBytes;
 #pragma unroll
-        for (int t = 0; t < kPass; ++t) {
-          if (t >= nt) continue;
-          const unsigned jt = j + t;
-          // this P^T buffer was last read by the value MMA of tile jt - NP
-          const int pb = jt % NP;
-          if (jt >= NP)
-            failed |= !wait_or_abort(&pv_done[pb], ((jt / NP) - 1) & 1, p.err, abort_flag, wl);
-          if constexpr (F8) {
-            // row h of P^T (K-major, 128 positions = 128 bytes, 128-byte swizzle): byte r
-            uint8_t* pt = smem + C::kOffP + pb * kPBytes;
+          for (int h = 0; h < G; h += 2) {
+            uint32_t hi, lo;
+            split_e4m3x2(pp[h], h + 1 < G ? pp[h + 1] : 0.f, kPLoScale, hi, lo);
 #pragma unroll
-            for (int h = 0; h < G; h += 2) {
-              uint32_t hi, lo;
-              split_e4m3x2(pp[t][h], h + 1 < G ? pp[t][h + 1] : 0.f, kPLoScale, hi, lo);
-#pragma unroll
-              for (int e = 0; e < 2 && h + e < G; ++e) {
-                const int hh = h + e;
-                const int off = hh * 128 + ((((r >> 4) ^ hh) & 7) << 4) + (r & 15);
-                pt[off] = static_cast<uint8_t>(hi >> (8 * e));
-                pt[kQRegion + off] = static_cast<uint8_t>(lo >> (8 * e));
-              }
-            }
-          } else {
-            uint8_t* pt = smem + C::kOffP + pb * kPBytes + (r >> 6) * kQRegion;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const int chunk = ((r & 63) >> 3) ^ (h & 7);
-              *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + chunk * 16 + (r & 7) * 2) =
-                  __float2bfloat16_rn(pp[t][h]);
+            for (int e = 0; e < 2 && h + e < G; ++e) {
+              const int hh = h + e;
+              const int off = hh * 128 + ((((r >> 4) ^ hh) & 7) << 4) + (r & 15);
+              pt[off] = static_cast<uint8_t>(hi >> (8 * e));
+              pt[kQRegion + off] = static_cast<uint8_t>(lo >> (8 * e));
             }
           }
-          if (i + t == d.ntiles - 1 && d.n - (i + t) * TM < TM) {
-            // V rows past the partition's end may hold anything (even NaN); P is 0
-            // there but 0 * NaN is NaN: clear them before the tensor core reads the tile
-            const int vs = jt % NV;
-            failed |= !wait_or_abort(&v_full[vs], (jt / NV) & 1, p.err, abort_flag, wl);
-            if (!valid[t]) {
-              uint8_t* v = smem + C::kOffV + vs * kTileBytes + r * 128;
+        } else {
+          uint8_t* pt = smem + C::kOffP + pb * kPBytes + (r >> 6) * kQRegion;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
-                if (!F8) *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
-              }
+          for (int h = 0; h < G; ++h) {
+            const int chunk = ((r & 63) >> 3) ^ (h & 7);
+            *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + chunk * 16 + (r & 7) * 2) =
+                __float2bfloat16_rn(pp[h]);
+          }
+        }
+        if (i == d.ntiles - 1 && d.n - i * TM < TM) {
+          // V rows past the partition's end may hold anything (even NaN); P is 0 there
+          // but 0 * NaN is NaN: clear them before the tensor core reads the tile
+          const int vs = j % NV;
+          failed |= !wait_or_abort(&v_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
+          if (!valid) {
+            uint8_t* v = smem + C::kOffV + vs * kTileBytes + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
+              if (!F8) *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
             }
           }
         }
-        if (rescale) {  // uniform across the group: every thread saw the same pair max
+        if (rescale) {  // uniform across the group: every thread saw the same tile max
           // O holds the value MMAs up to tile j-1: wait for the last of them
           const unsigned t = j - 1;
           failed |= !wait_or_abort(&pv_done[t % NP], (t / NP) & 1, p.err, abort_flag, wl);
@@ -1195,11 +1126,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&p_full[j % NP]);
-          if (nt == 2) mbar_arrive(&p_full[(j + 1) % NP]);
-        }
-        j += nt;
+        if (lane == 0) mbar_arrive(&p_full[pb]);
       }
       // hand the item to the epilogue warps: l per head (the per-position shares summed
       // over the 128 threads), the reference max and, for e4m3, O's factor 2^(R - m);
