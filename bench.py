@@ -353,8 +353,9 @@ def measure_fp8_decode(torch, pa, hbm_peak, peak_src, bf16_attn_us, steps=200, w
     a_ms = sum(attn_ms) / len(attn_ms)
     st_ms = total_ms / steps - a_ms
     b = fp8_decode_bytes(w)
-    d = {"kernel": "pa_decode_fp8 (persistent tcgen05 decode, e4m3 tiles dequantised in "
-                   "shared memory)", "attn_us": round(a_ms * 1e3, 2),
+    d = {"kernel": "pa_decode_fp8 (persistent tcgen05 decode; kind::f8f6f4 MMAs read the "
+                   "stored e4m3 codes, row scales applied in the softmax)",
+         "attn_us": round(a_ms * 1e3, 2),
          "step_us": round(total_ms / steps * 1e3, 2), "steps": steps, "launches_per_step": lps,
          "algorithmic_bytes": b, "GBps": round(b / a_ms / 1e6, 1),
          "frac_of_hbm_peak": round(b / a_ms / 1e6 / hbm_peak, 3),

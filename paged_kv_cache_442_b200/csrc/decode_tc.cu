@@ -313,16 +313,6 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
   for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 2-D tiled tensor load global -> shared (the fp8 scales: [Hkv][slots] fp32).
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -551,60 +541,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       if (!F8) kq = k + 1;
       ++npub;
       bool alive = true;
+      __syncwarp();  // converged: the loop's loads are elected from the whole warp
+      // The whole warp runs the tile loop (waits and coordinates warp-uniform); one
+      // elected lane issues each load. A lane-0 branch with broadcast verdicts cost this
+      // warp ~2000 cycles a tile, more than an e4m3 tile's share of the DRAM time.
       for (int i = 0; i < ntiles; ++i) {
         // K of tile jk: its slot frees when the score MMA of tile jk - NK is done
         const int ks = jk % NK;
-        if (jk >= NK && !wwait(&k_empty[ks], ((jk / NK) - 1) & 1)) {
+        if (jk >= NK && !warp_wait_or_abort(&k_empty[ks], ((jk / NK) - 1) & 1, p.err, abort_flag, wl)) {
           alive = false;
           break;
         }
         const int kl = F8 ? jk % NSC : 0;
-        if (F8 && jk >= NSC && !wwait(&ksc_empty[kl], ((jk / NSC) - 1) & 1)) {
+        if (F8 && jk >= NSC &&
+            !warp_wait_or_abort(&ksc_empty[kl], ((jk / NSC) - 1) & 1, p.err, abort_flag, wl)) {
           alive = false;
           break;
         }
-        if (lane == 0) {
+        {
           uint8_t* kdst = smem + C::kOffK + ks * kTileBytes;
-          mbar_arrive_expect_tx(&k_full[ks], kTileBytes);
-          if (F8) mbar_arrive_expect_tx(&ksc_full[kl], TM * 4);
+          mbar_arrive_expect_tx_w(&k_full[ks], kTileBytes);
+          if (F8) mbar_arrive_expect_tx_w(&ksc_full[kl], TM * 4);
           for (int b = 0; b < nbox; ++b) {
             const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
             if (F8) {
-              tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
-              tma_load_2d(smem + C::kOffScl + kl * kSclBytes + b * sstride, &tmSK, &ksc_full[kl],
-                          row, g);
+              tma_load_3d_w(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
+              tma_load_2d_w(smem + C::kOffScl + kl * kSclBytes + b * sstride, &tmSK, &ksc_full[kl],
+                            row, g);
             } else {
-              tma_load_3d(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
-              tma_load_3d(kdst + kRegion + b * rows * 128, &tmK, &k_full[ks], 64, g, row);
+              tma_load_3d_w(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
+              tma_load_3d_w(kdst + kRegion + b * rows * 128, &tmK, &k_full[ks], 64, g, row);
             }
           }
         }
         ++jk;
-        __syncwarp();
         // V of tile jv: its slot frees when the value MMA of tile jv - NV is done
         const int vs = jv % NV;
-        if (jv >= NV && !wwait(&v_empty[vs], ((jv / NV) - 1) & 1)) {
+        if (jv >= NV && !warp_wait_or_abort(&v_empty[vs], ((jv / NV) - 1) & 1, p.err, abort_flag, wl)) {
           alive = false;
           break;
         }
-        if (lane == 0) {
+        {
           uint8_t* vdst = smem + C::kOffV + vs * kTileBytes;
-          mbar_arrive_expect_tx(&v_full[vs], kTileBytes);
-          if (F8) mbar_arrive_expect_tx(&vsc_full[vs], TM * 4);
+          mbar_arrive_expect_tx_w(&v_full[vs], kTileBytes);
+          if (F8) mbar_arrive_expect_tx_w(&vsc_full[vs], TM * 4);
           for (int b = 0; b < nbox; ++b) {
             const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
             if (F8) {
-              tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
-              tma_load_2d(smem + C::kOffScl + (NSC + vs) * kSclBytes + b * sstride, &tmSV,
-                          &vsc_full[vs], row, g);
+              tma_load_3d_w(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
+              tma_load_2d_w(smem + C::kOffScl + (NSC + vs) * kSclBytes + b * sstride, &tmSV,
+                            &vsc_full[vs], row, g);
             } else {
-              tma_load_3d(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
-              tma_load_3d(vdst + kRegion + b * rows * 128, &tmV, &v_full[vs], 64, g, row);
+              tma_load_3d_w(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
+              tma_load_3d_w(vdst + kRegion + b * rows * 128, &tmV, &v_full[vs], 64, g, row);
             }
           }
         }
         ++jv;
-        __syncwarp();
       }
       if (!alive) break;
       if (lane == 0) mbar_arrive(&sched_empty[ss]);  // this item's block ids are no longer needed
