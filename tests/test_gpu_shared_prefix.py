@@ -98,3 +98,22 @@ def test_shared_prefix_reports_a_table_without_the_shared_blocks():
     with pytest.raises(pa.PAError) as e:
         shared_decode(dw, 1024, blocks=shared_blocks_of(w, 1024), bt=i32_dev(bt))
     assert e.value.status == 3
+
+
+def test_shared_prefix_two_units_per_cta():
+    """A batch large enough that the prefix pass runs two 128-row units per CTA (with 16
+    query heads per kv head a unit holds 8 sequences; 320 sequences x 8 kv heads fill
+    more than one unit per SM), checked against the oracle on sampled sequences,
+    contexts shorter than, equal to and just past the prefix among them."""
+    S = 128
+    rng = np.random.default_rng(21)
+    lens = rng.integers(1, 420, size=320)
+    lens[:4] = [1, 127, 128, 129]
+    w = build_workload(kind="decode", context_lens=lens, new_lens=np.ones_like(lens),
+                       num_q_heads=128, num_kv_heads=8, head_dim=128, block_size=64,
+                       seed=2100, shared_prefix_len=S)
+    dw = DeviceWorkload(w)
+    out = to_f64(shared_decode(dw, S))
+    seqs = np.unique(np.concatenate([np.arange(6), rng.choice(w.num_seqs, size=18, replace=False),
+                                     [w.num_seqs - 1]]))
+    assert_close(out[seqs], oracle_decode(w, seqs=seqs), "two units per CTA (sampled)")
