@@ -399,9 +399,10 @@ pa_status pa_store_kvcache_fp8(const void* k, const void* v, void* k_codes, void
  * pools hold (code * scale). The tensor cores read the stored codes directly
  * (e4m3 x e4m3 products, fp32 accumulation); no code is converted. Each row's K
  * scale multiplies that position's score, and each row's V scale its probability,
- * in fp32. q and the probabilities reach the tensor cores as two e4m3 terms each
- * (a high term and the rounded remainder), which keeps about 2^-8 relative
- * accuracy per element. Arguments as pa_decode, with the pools replaced by codes
+ * in fp32. q reaches the tensor cores as three e4m3 terms (about 2^-13 relative
+ * per element: a score's error is multiplied by the score's size in the exponent,
+ * so peaked softmaxes need q this exact) and the probabilities as two (a high term
+ * and the scaled remainder: about 2^-8 relative per element). Arguments as pa_decode, with the pools replaced by codes
  * and scales (16-byte aligned). Values whose products overflow fp32 are out of
  * range (as for pa_decode).
  * Supported: head_dim 128, Hq / Hkv in {1, 2, 4, 8, 16}, partition_size (given or

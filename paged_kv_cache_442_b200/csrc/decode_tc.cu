@@ -14,20 +14,22 @@
 //   warp 10 scheduler: takes the next item from the counter, skips empty partitions
 //           (writing zero rows for empty contexts) and reads the item's block ids, one
 //           item ahead of the producer;
-//   warp 4  producer: loads q (one box per item) and the K and V tiles
-//           of 128 positions through the block table (one TMA box per physical
-//           block) into a K ring and a V ring. A K slot frees as soon as its score
-//           MMA is done and a V slot when its value MMA is done, so both streams run
-//           several tiles ahead of the consumers (the fetch latency, ~1.4 us per tile,
-//           must overlap);
+//   warp 4  producer: loads q (bf16: one box per item) and the K and V tiles of 128
+//           positions through the block table (one TMA box per physical block) into a
+//           K ring and a V ring; the whole warp waits and computes the coordinates, an
+//           elected lane issues each load. A K slot frees as soon as its score MMA is
+//           done and a V slot when its value MMA is done, so both streams run several
+//           tiles ahead of the consumers (the fetch latency, ~1.4 us per tile, must
+//           overlap);
 //   warp 5  tensor-core issuer: owns the TMEM allocation; an event loop over two
 //           cursors: the value MMA O^T += V^T P^T of the oldest scored tile whenever its
 //           P, V and accumulator are ready (the softmax and the V ring wait on it),
 //           else the score MMA S^T of the next tile, up to four tiles ahead and across
-//           item boundaries, whenever its item, K tile and S buffer are ready. Every
-//           issue group costs the issuing warp several hundred cycles, so the order
-//           matters: value first keeps V slots and P buffers turning over, and scoring
-//           ahead lets the next item's first tile be ready when the softmax gets there;
+//           item boundaries, whenever its item, K tile and S buffer are ready. In the
+//           kernel an issue group with its waits and commits takes the warp several
+//           hundred cycles, so the order matters: value first keeps V slots and P
+//           buffers turning over, and scoring ahead lets the next item's first tile be
+//           ready when the softmax gets there;
 //   warps 0-3  softmax: thread r owns position r of a tile (TMEM lane r): per-head
 //           tile max across the 128 positions, exp2 against a per-item reference max,
 //           P^T to shared memory. O^T is rescaled in TMEM only when a tile's max
@@ -62,8 +64,7 @@
 //     operand, so one product fills two side-by-side O^T accumulators combined as
 //     O_hi + O_lo / 128 (about 2^-8 relative on P', and an absolute floor near 2^-17,
 //     so small probabilities keep their precision).
-// Per tile that is 4 + 4 MMA instructions (K = 32 bytes each): the single issuing
-// thread, not the tensor core, sets the pace of small products like these.
+// Per tile that is 4 + 4 MMA instructions (K = 32 bytes each) instead of 20.
 // Before a CTA ends, its producer waits for every copy it started and its issuer for
 // every MMA it issued (with the full time limit, even when the roles gave up early),
 // so no asynchronous write outlives the CTA's shared and tensor memory.
@@ -631,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // counter), skips empty partitions, reads the context length and the item's
     // block ids, and queues them for the producer QS deep, so none of these dependent
     // global reads sit on the TMA producer's path. For e4m3 pools it also writes the
-    // item's q as two e4m3 terms into the item's Q slot.
+    // item's q as three e4m3 terms into the item's Q slot.
     int q = 0;
     bool first_take = true;
     while (true) {

@@ -1,4 +1,5 @@
-"""The FMA-pipe exponential of the kernels (ex2_poly2 in csrc/pa_ptx.cuh), checked on
+"""The FMA-pipe exponential (ex2_poly2 in csrc/pa_ptx.cuh; no kernel calls it, it
+measured slower than ex2.approx in the prefill softmax), checked on
 the CPU: its coefficients are read out of the header, its steps (range reduction by the
 1.5 * 2^23 shift, degree-3 polynomial by fused multiply-adds, exponent added to the
 bits) are replayed in float32, and the result is compared with the exact 2^x.

@@ -3,9 +3,10 @@
 Store: codes and scales bit-exact against the oracle's quantiser (both take every
 decision in fp32 with round-to-nearest). Decode: within the decode bar of
 tests/gpu_helpers.py against the oracle's fp64 attention of the exact values the pools
-hold (code * scale). The kernel's tensor cores read the codes themselves (exact); q and
-the probabilities reach them as two e4m3 terms each (about 2^-8 relative error per
-element, of the size of the bf16 rounding of P that the bf16 decode carries).
+hold (code * scale). The kernel's tensor cores read the codes themselves (exact); q
+reaches them as three e4m3 terms (about 2^-13 relative per element) and the
+probabilities as two (about 2^-8 relative, of the size of the bf16 rounding of P that
+the bf16 decode carries).
 """
 import numpy as np
 import pytest
@@ -225,9 +226,9 @@ def test_fp8_decode_agrees_with_bf16_decode_on_exact_rows():
     """Rows that are e4m3 values times a power of two survive quantising exactly, and
     their dequantised values are exact in bf16: the fp8 and bf16 decodes then attend
     over the same numbers. They round differently on the way (the fp8 kernel feeds q
-    and the probabilities to the tensor cores as two e4m3 terms each, the bf16 kernel
-    rounds the probabilities to bf16), so both are checked against the oracle and
-    against each other to a tight norm."""
+    to the tensor cores as three e4m3 terms and the probabilities as two, the bf16
+    kernel rounds the probabilities to bf16), so both are checked against the oracle
+    and against each other to a tight norm."""
     lens = np.array([40, 300, 1, 129])
     w = build_workload(kind="decode", context_lens=lens, new_lens=np.ones(4, int), num_q_heads=8,
                        num_kv_heads=2, head_dim=128, block_size=16, seed=812)
