@@ -211,3 +211,23 @@ def test_bad_block_id_is_reported_not_faulted():
         pa.pa_set_debug_checks(True)
     # the context stays usable
     assert_close(to_f64(dw.decode()), oracle_decode(w), "after bad index")
+
+
+@pytest.mark.parametrize("P", [0, 128])
+def test_decode_many_one_tile_items(P):
+    """640 sequences of at most 130 positions over 8 kv heads: thousands of work items of
+    one or two tiles, so the tensor-core issuer crosses an item boundary at almost every
+    tile (its score cursor runs ahead across items) and each CTA runs dozens of items,
+    reusing every item slot, S buffer, P buffer and O accumulator many times."""
+    rng = np.random.default_rng(64)
+    lens = rng.integers(1, 131, size=640)
+    lens[:6] = [1, 2, 127, 128, 129, 130]
+    w = build_workload(kind="decode", context_lens=lens, new_lens=np.ones_like(lens),
+                       num_q_heads=16, num_kv_heads=8, head_dim=128, block_size=16,
+                       seed=6400 + P)
+    dw = DeviceWorkload(w)
+    got = to_f64(dw.decode(P))
+    assert_close(got, oracle_decode(w), f"one-tile items P={P}")
+    # and the same bits when the batch is decoded again (every item slot reused)
+    again = to_f64(dw.decode(P))
+    assert np.array_equal(got, again)

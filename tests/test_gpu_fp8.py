@@ -292,3 +292,17 @@ def test_fp8_decode_zero_rows_and_zero_queries():
         got = gpu_decode_fp8(w, pools, P)
         assert_close(got, oracle_decode_fp8(w, pools.host), f"zero rows P={P}")
         assert np.all(got[3] == 0)
+
+
+def test_fp8_decode_many_one_tile_items():
+    """e4m3 pools, 640 sequences of at most 130 positions over 8 kv heads: an item
+    boundary at almost every tile for the issuer, the scheduler's q terms and the
+    K-scale ring."""
+    rng = np.random.default_rng(65)
+    lens = rng.integers(1, 131, size=640)
+    lens[:6] = [1, 2, 127, 128, 129, 130]
+    w = build_workload(kind="decode", context_lens=lens, new_lens=np.ones_like(lens),
+                       num_q_heads=16, num_kv_heads=8, head_dim=128, block_size=16, seed=6500)
+    pools = Fp8Pools(w)
+    got = gpu_decode_fp8(w, pools, 128)
+    assert_close(got, oracle_decode_fp8(w, pools.host), "fp8 one-tile items")
