@@ -82,7 +82,7 @@
 namespace pa {
 namespace {
 
-constexpr int TM = 128;        // positions per tile
+constexpr int TM = 128;        // positions per product (the MMAs' M) and per bf16 tile
 constexpr int HD = 128;        // head dim
 constexpr int NQ = 16;         // MMA N: query heads of one kv head, padded
 constexpr int NS = 4;          // S^T buffers in TMEM
@@ -95,9 +95,12 @@ constexpr int kThreads = 352;  // softmax 0-3, producer 4, issuer 5, epilogue 6-
 constexpr float kRescaleLog2 = 8.f;  // rescale when the max grows by more than this
 constexpr int kQRegion = NQ * 128;           // 16 rows x 128 bytes (2 KB)
 constexpr int kQTerms = 3;                   // e4m3: q as hi + mid + lo terms
-constexpr int kPBytes = 2 * kQRegion;        // bf16: P^T 16 x 128; e4m3: hi, lo terms
+constexpr int kPChunk = 2 * kQRegion;        // bf16: P^T 16 x 128; e4m3: hi, lo terms of 128 positions
 constexpr int kMaxIds = 2048 / 16 + 2;       // block ids of one item (partition <= 2048)
-constexpr int kSclBytes = 1024;              // e4m3: one tile's row scales (<= 8 boxes)
+// e4m3: one tile's 256 row scales: one box per physical block, each box on a 128-byte
+// boundary (a tensor copy's shared-memory destination must be 128-byte aligned), so 16
+// boxes of 16 scales (block size 16) take 2 KB
+constexpr int kSclBytes = 2048;
 constexpr int kEpiBytes = 32 + 3 * NQ * 4;   // descriptor, m, l, e4m3 output factor
 // e4m3 value path: P' <= 2^kPBoundLog2 (a rescale brings the bound to 2^kPTargetLog2),
 // so its low term, scaled by kPLoScale, stays inside e4m3's range (|128 (P' - hi)| <=
@@ -113,11 +116,18 @@ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 // the static_asserts below keep it that way when depths change.
 template <bool F8>
 struct Cfg {
+  // A tile is 128 positions of bf16 rows (256 bytes each) or 256 positions of e4m3 rows
+  // (128 bytes each): 32 KB either way. Every tile costs the kernel's roles about the
+  // same time whatever it holds, so e4m3 tiles of 128 positions (16 KB) left the e4m3
+  // decode at half the bf16 decode's bandwidth.
+  static constexpr int TT = F8 ? 2 * TM : TM;                 // positions per tile
+  static constexpr int kSub = TT / TM;                         // products of 128 positions
   static constexpr int kRegion = TM * 128;                    // 128 rows x 128 bytes
-  static constexpr int kTileBytes = F8 ? kRegion : 2 * kRegion;  // one K or V tile
-  static constexpr int NK = F8 ? 5 : 3;  // K ring (a slot frees when its score MMA is done)
-  static constexpr int NV = F8 ? 6 : 3;  // V ring (a slot frees when its value MMA is done)
-  static constexpr int NSC = F8 ? 8 : 1;  // e4m3: K-scale ring (freed by the softmax); unused for bf16
+  static constexpr int kTileBytes = 2 * kRegion;              // one K or V tile
+  static constexpr int NK = F8 ? 2 : 3;  // K ring (a slot frees when its score MMA is done)
+  static constexpr int NV = 3;           // V ring (a slot frees when its value MMA is done)
+  static constexpr int NSC = F8 ? 4 : 1;  // e4m3: K-scale ring (freed by the softmax); unused for bf16
+  static constexpr int kPBytes = kSub * kPChunk;  // one P^T buffer
   static constexpr int kQBytes = (F8 ? kQTerms : 2) * kQRegion;  // bf16: two 64-dim halves
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + NK * kTileBytes;
@@ -135,14 +145,14 @@ struct Cfg {
   static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * QN + 2 * NS + 2 * NP + 4 * NO + 2 * QS +
                                   1 + (F8 ? 2 * NSC + NV + QN : 0);
   static constexpr int kOffMisc = align_up(kOffBar + 8 * kNumBars, 16);
-  // e4m3: the K-scale ring [NSC] and each V slot's scales [NV], 1 KB each
+  // e4m3: the K-scale ring [NSC] and each V slot's scales [NV], kSclBytes each
   static constexpr int kOffScl = align_up(kOffMisc + 64, 1024);
   static constexpr int kSmemBytes = (F8 ? kOffScl + (NSC + NV) * kSclBytes : kOffMisc + 64) + 1024;
-  // TMEM columns. bf16: S^T[NS] 16 columns each, then O^T[NO] 16 each. e4m3: S^T[NS] 48
-  // columns each (the hi, mid and lo q terms' products side by side: one MMA with the
-  // three terms stacked as N = 48), then O^T[NO] 32 each (P's hi and lo terms stacked as
-  // N = 32: the hi accumulator, then the lo one)
-  static constexpr uint32_t kSCols = F8 ? NQ * kQTerms : NQ;
+  // TMEM columns. bf16: S^T[NS] 16 columns each, then O^T[NO] 16 each. e4m3: S^T[NS] 96
+  // columns each (per 128 positions, the hi, mid and lo q terms' products side by side:
+  // one MMA with the three terms stacked as N = 48; two such for a tile), then O^T[NO]
+  // 32 each (P's hi and lo terms stacked as N = 32: the hi accumulator, then the lo one)
+  static constexpr uint32_t kSCols = F8 ? kSub * NQ * kQTerms : NQ;
   static constexpr uint32_t kOCols = F8 ? 2 * NQ : NQ;
   static constexpr uint32_t kTmemO = NS * kSCols;
   static constexpr uint32_t kTmemCols = F8 ? 512 : 128;
@@ -397,12 +407,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
-  // e4m3: where a tile's row scales sit (box r / rows, each box on a 128-byte boundary)
-  const int srows = bs < TM ? bs : TM;
+  // e4m3: where a tile's row scales sit (box r / rows, each box on a 128-byte boundary:
+  // a tensor copy's shared-memory destination must be 128-byte aligned)
+  const int srows = bs < C::TT ? bs : C::TT;
   const int sstride = srows * 4 < 128 ? 128 : srows * 4;
 
   // zero the Q slots and P^T buffers: rows >= G are never written and stay zero
-  for (int i = tid; i < (QN * C::kQBytes + NP * kPBytes) / 16; i += blockDim.x)
+  for (int i = tid; i < (QN * C::kQBytes + NP * C::kPBytes) / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + C::kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
@@ -475,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   if (warp == 4) {
     // ======================================================== producer warp
     const int rows = srows;
-    const int nbox = TM / rows;
+    const int nbox = C::TT / rows;
     int q = 0;        // items taken from the scheduler queue
     int k = 0;        // items published to the issuer / softmax
     int kq = 0;       // q loads started (bf16)
@@ -562,9 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         {
           uint8_t* kdst = smem + C::kOffK + ks * kTileBytes;
           mbar_arrive_expect_tx_w(&k_full[ks], kTileBytes);
-          if (F8) mbar_arrive_expect_tx_w(&ksc_full[kl], TM * 4);
+          if (F8) mbar_arrive_expect_tx_w(&ksc_full[kl], C::TT * 4);
           for (int b = 0; b < nbox; ++b) {
-            const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
+            const int row = row_of(idc, first_blk, t0 + i * C::TT + b * rows);
             if (F8) {
               tma_load_3d_w(kdst + b * rows * 128, &tmK, &k_full[ks], 0, g, row);
               tma_load_2d_w(smem + C::kOffScl + kl * kSclBytes + b * sstride, &tmSK, &ksc_full[kl],
@@ -585,9 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         {
           uint8_t* vdst = smem + C::kOffV + vs * kTileBytes;
           mbar_arrive_expect_tx_w(&v_full[vs], kTileBytes);
-          if (F8) mbar_arrive_expect_tx_w(&vsc_full[vs], TM * 4);
+          if (F8) mbar_arrive_expect_tx_w(&vsc_full[vs], C::TT * 4);
           for (int b = 0; b < nbox; ++b) {
-            const int row = row_of(idc, first_blk, t0 + i * TM + b * rows);
+            const int row = row_of(idc, first_blk, t0 + i * C::TT + b * rows);
             if (F8) {
               tma_load_3d_w(vdst + b * rows * 128, &tmV, &v_full[vs], 0, g, row);
               tma_load_2d_w(smem + C::kOffScl + (NSC + vs) * kSclBytes + b * sstride, &tmSV,
@@ -678,9 +689,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           continue;
         }
         const int n = min(ctx - t0, p.partition_size);
-        const int ntiles = (n + TM - 1) / TM;
+        const int ntiles = (n + C::TT - 1) / C::TT;
         first_blk = t0 >> p.bs_log2;
-        const int nb = ((t0 + ntiles * TM - 1) >> p.bs_log2) - first_blk + 1;
+        const int nb = ((t0 + ntiles * C::TT - 1) >> p.bs_log2) - first_blk + 1;
         int* idb = ids + slot * kMaxIds;
         for (int i = lane; i < nb && i < kMaxIds; i += 32) {
           const int b = first_blk + i;
@@ -798,12 +809,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         const uint64_t aK = smem_desc_sw128(smem_u32(smem + C::kOffK + kslot * kTileBytes), 16, 1024);
         const uint64_t bQ = smem_desc_sw128(sQ, 16, 1024);
         if (F8) {
-          // [K hi^T | K mid^T | K lo^T] in one product: the three q terms are the 48 rows
-          // of one B operand; 32 head dims (bytes) of each row per instruction
+          // per 128 positions, [K hi^T | K mid^T | K lo^T] in one product: the three q
+          // terms are the 48 rows of one B operand; 32 head dims (bytes) of each row per
+          // instruction; positions 128 h .. 128 h + 127 (rows of the tile 16 KB apart)
+          // into columns 48 h .. 48 h + 47 of the S buffer
 #pragma unroll
-          for (int kk = 0; kk < HD / 32; ++kk)
-            tc_mma_f8_ss(tmem + sb * C::kSCols, desc_advance(aK, kk * 32),
-                         desc_advance(bQ, kk * 32), idS, kk > 0 ? 1u : 0u);
+          for (int h = 0; h < C::kSub; ++h)
+#pragma unroll
+            for (int kk = 0; kk < HD / 32; ++kk)
+              tc_mma_f8_ss(tmem + sb * C::kSCols + h * NQ * kQTerms,
+                           desc_advance(aK, h * kRegion + kk * 32), desc_advance(bQ, kk * 32), idS,
+                           kk > 0 ? 1u : 0u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
@@ -837,14 +853,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         // one descriptor per operand, stepped by constant offsets (see desc_advance)
         const uint64_t aV = smem_desc_sw128(smem_u32(smem + C::kOffV + vs * kTileBytes),
                                             kRegion, 1024);
-        const uint64_t bP = smem_desc_sw128(sP + b * kPBytes, 16, 1024);
+        const uint64_t bP = smem_desc_sw128(sP + b * C::kPBytes, 16, 1024);
         const uint32_t dO = tmem + C::kTmemO + obuf * C::kOCols;
         if (F8) {
           // 32 positions (4 rows of 8-row swizzle atoms) per instruction; P's hi and lo
-          // terms are one B operand of 32 rows, so O_hi and O_lo come out side by side
+          // terms are one B operand of 32 rows (per 128 positions: a chunk of P^T), so
+          // O_hi and O_lo come out side by side
 #pragma unroll
-          for (int kk = 0; kk < TM / 32; ++kk)
-            tc_mma_f8_ss(dO, desc_advance(aV, kk * 32 * 128), desc_advance(bP, kk * 32), idO,
+          for (int kk = 0; kk < C::TT / 32; ++kk)
+            tc_mma_f8_ss(dO, desc_advance(aV, kk * 32 * 128),
+                         desc_advance(bP, (kk >> 2) * kPChunk + (kk & 3) * 32), idO,
                          (first && kk == 0) ? 0u : 1u);
         } else {
 #pragma unroll
@@ -909,8 +927,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // at a named barrier.
     const int r = tid;  // position within a tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    // e4m3: byte offset of position r's scale within a tile's scale area
-    const int soff = (r / srows) * sstride + (r % srows) * 4;
+    // e4m3: byte offsets of this thread's positions' scales within a tile's scale area
+    int soff[C::kSub];
+#pragma unroll
+    for (int u = 0; u < C::kSub; ++u) {
+      const int pos = u * TM + r;
+      soff[u] = (pos / srows) * sstride + (pos % srows) * 4;
+    }
     int k = 0;
     unsigned j = 0;  // tiles of this CTA done
     while (true) {
@@ -944,62 +967,87 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         lp[h] = 0.f;
         R[h] = -INFINITY;  // e4m3: O's reference, unset until a tile has a non-zero V scale
       }
+      // A tile is SUB products of 128 positions: thread r owns position r of each
+      // (r and 128 + r for e4m3 tiles of 256).
+      constexpr int SUB = C::kSub;
       for (int i = 0; i < d.ntiles; ++i, ++j) {
         const int sb = j % NS;
-        const bool valid = i * TM + r < d.n;
+        bool valid[SUB];
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) valid[u] = i * C::TT + u * TM + r < d.n;
         // e4m3: the tile's K and V row scales first: they land with the tiles, well
         // before the score MMA is done, so their waits and reads overlap it
-        float skr = 1.f;
-        float svr = 0.f;  // e4m3: this position's V scale (0 past the partition)
+        float skr[SUB], svr[SUB];  // svr: this position's V scale (0 past the partition)
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) {
+          skr[u] = 1.f;
+          svr[u] = 0.f;
+        }
         if constexpr (F8) {
           const int kl = j % NSC;
           failed |= !wait_or_abort(&ksc_full[kl], (j / NSC) & 1, p.err, abort_flag, wl);
-          skr = *reinterpret_cast<const float*>(smem + C::kOffScl + kl * kSclBytes + soff);
+#pragma unroll
+          for (int u = 0; u < SUB; ++u)
+            skr[u] = *reinterpret_cast<const float*>(smem + C::kOffScl + kl * kSclBytes + soff[u]);
           __syncwarp();
           if (lane == 0) mbar_arrive(&ksc_empty[kl]);
           const int vs = j % NV;
           failed |= !wait_or_abort(&vsc_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
-          if (valid)
-            svr = *reinterpret_cast<const float*>(smem + C::kOffScl + (NSC + vs) * kSclBytes + soff);
+#pragma unroll
+          for (int u = 0; u < SUB; ++u)
+            if (valid[u])
+              svr[u] = *reinterpret_cast<const float*>(smem + C::kOffScl + (NSC + vs) * kSclBytes +
+                                                       soff[u]);
         }
         failed |= !wait_or_abort(&s_full[sb], (j / NS) & 1, p.err, abort_flag, wl);
         tc_fence_after();
-        float sv[G];
-        tmem_ld_cols<G>(tmem + sb * C::kSCols + lane_off, sv);
-        if constexpr (F8) {
-          // S = products with the hi, mid and lo q terms, summed
-          float s1[G], s2[G];
-          tmem_ld_cols<G>(tmem + sb * C::kSCols + NQ + lane_off, s1);
-          tmem_ld_cols<G>(tmem + sb * C::kSCols + 2 * NQ + lane_off, s2);
-          tc_wait_ld();
+        float sv[SUB][G];
 #pragma unroll
-          for (int h = 0; h < G; ++h) sv[h] = (sv[h] + s1[h]) + s2[h];
+        for (int u = 0; u < SUB; ++u) {
+          const uint32_t ts = tmem + sb * C::kSCols + u * NQ * kQTerms + lane_off;
+          tmem_ld_cols<G>(ts, sv[u]);
+          if constexpr (F8) {
+            // S = products with the hi, mid and lo q terms, summed
+            float s1[G], s2[G];
+            tmem_ld_cols<G>(ts + NQ, s1);
+            tmem_ld_cols<G>(ts + 2 * NQ, s2);
+            tc_wait_ld();
+#pragma unroll
+            for (int h = 0; h < G; ++h) sv[u][h] = (sv[u][h] + s1[h]) + s2[h];
+          }
         }
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
-        float x[G];
-        if constexpr (F8) {
-          const float fr = p.scale_log2 * skr;
+        float x[SUB][G];
 #pragma unroll
-          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * (fr * qsg[h]) : -INFINITY;
-        } else {
+        for (int u = 0; u < SUB; ++u) {
+          if constexpr (F8) {
+            const float fr = p.scale_log2 * skr[u];
 #pragma unroll
-          for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+            for (int h = 0; h < G; ++h) x[u][h] = valid[u] ? sv[u][h] * (fr * qsg[h]) : -INFINITY;
+          } else {
+#pragma unroll
+            for (int h = 0; h < G; ++h) x[u][h] = valid[u] ? sv[u][h] * p.scale_log2 : -INFINITY;
+          }
         }
         // per-head max over the tile: warp shuffles, then across the 4 warps
         float* rb = red + (j & 1) * 4 * NQ;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          float v = x[h];
+          float v = x[0][h];
+#pragma unroll
+          for (int u = 1; u < SUB; ++u) v = fmaxf(v, x[u][h]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) rb[warp * NQ + h] = v;
         }
         float* svb = red + 3 * 4 * NQ + (j & 1) * 4;  // e4m3: the tile's largest V scale
         if (F8) {
-          float v = svr;
+          float v = svr[0];
+#pragma unroll
+          for (int u = 1; u < SUB; ++u) v = fmaxf(v, svr[u]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) svb[warp] = v;
@@ -1007,11 +1055,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         named_bar_sync(1, 128);
         bool rescale = false;
         float alpha[G];
-        float pp[G];  // e4m3: P' of this position per head
+        float pp[SUB][G];  // P' (e4m3) or P (bf16) of this thread's positions per head
         if constexpr (F8) {
           // bound of P' over the tile: 2^(max x + log2 max s_v - R)
           const float lsm = lg2_approx(fmaxf(fmaxf(svb[0], svb[1]), fmaxf(svb[2], svb[3])));
-          const float lsv = lg2_approx(svr);  // -inf for s_v = 0 (and past the partition)
+          float lsv[SUB];
+#pragma unroll
+          for (int u = 0; u < SUB; ++u) lsv[u] = lg2_approx(svr[u]);  // -inf for s_v = 0
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
@@ -1022,8 +1072,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
               lp[h] *= ex2_approx(m[h] - mx);
               m[h] = mx;
             }
-            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
-            lp[h] += pr;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) lp[h] += valid[u] ? ex2_approx(x[u][h] - m[h]) : 0.f;
             // O's reference: set by the first tile with a non-zero V scale (O is exactly
             // 0 before it), raised when the bound would pass 2^kPBoundLog2
             alpha[h] = 1.f;
@@ -1036,7 +1086,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
               R[h] = rn;
               rescale = true;
             }
-            pp[h] = (valid && R[h] > -INFINITY) ? ex2_approx(x[h] + lsv - R[h]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u)
+              pp[u][h] = (valid[u] && R[h] > -INFINITY) ? ex2_approx(x[u][h] + lsv[u] - R[h]) : 0.f;
           }
         } else {
 #pragma unroll
@@ -1050,9 +1102,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
               m[h] = mx;
               rescale = true;
             }
-            const float pr = valid ? ex2_approx(x[h] - m[h]) : 0.f;
-            lp[h] = lp[h] * alpha[h] + pr;
-            pp[h] = pr;
+            float ps = 0.f;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) {
+              pp[u][h] = valid[u] ? ex2_approx(x[u][h] - m[h]) : 0.f;
+              ps += pp[u][h];
+            }
+            lp[h] = lp[h] * alpha[h] + ps;
           }
         }
         // this P^T buffer was last read by the value MMA of tile j - NP
@@ -1060,40 +1116,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (j >= NP)
           failed |= !wait_or_abort(&pv_done[pb], ((j / NP) - 1) & 1, p.err, abort_flag, wl);
         if constexpr (F8) {
-          // row h of P^T (K-major, 128 positions = 128 bytes, 128-byte swizzle): byte r
-          uint8_t* pt = smem + C::kOffP + pb * kPBytes;
+          // row h of P^T (K-major, 128 positions = 128 bytes per chunk, 128-byte
+          // swizzle): byte r of chunk u; the lo terms kQRegion after the hi ones
 #pragma unroll
-          for (int h = 0; h < G; h += 2) {
-            uint32_t hi, lo;
-            split_e4m3x2(pp[h], h + 1 < G ? pp[h + 1] : 0.f, kPLoScale, hi, lo);
+          for (int u = 0; u < SUB; ++u) {
+            uint8_t* pt = smem + C::kOffP + pb * C::kPBytes + u * kPChunk;
 #pragma unroll
-            for (int e = 0; e < 2 && h + e < G; ++e) {
-              const int hh = h + e;
-              const int off = hh * 128 + ((((r >> 4) ^ hh) & 7) << 4) + (r & 15);
-              pt[off] = static_cast<uint8_t>(hi >> (8 * e));
-              pt[kQRegion + off] = static_cast<uint8_t>(lo >> (8 * e));
+            for (int h = 0; h < G; h += 2) {
+              uint32_t hi, lo;
+              split_e4m3x2(pp[u][h], h + 1 < G ? pp[u][h + 1] : 0.f, kPLoScale, hi, lo);
+#pragma unroll
+              for (int e = 0; e < 2 && h + e < G; ++e) {
+                const int hh = h + e;
+                const int off = hh * 128 + ((((r >> 4) ^ hh) & 7) << 4) + (r & 15);
+                pt[off] = static_cast<uint8_t>(hi >> (8 * e));
+                pt[kQRegion + off] = static_cast<uint8_t>(lo >> (8 * e));
+              }
             }
           }
         } else {
-          uint8_t* pt = smem + C::kOffP + pb * kPBytes + (r >> 6) * kQRegion;
+          uint8_t* pt = smem + C::kOffP + pb * C::kPBytes + (r >> 6) * kQRegion;
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const int chunk = ((r & 63) >> 3) ^ (h & 7);
             *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + chunk * 16 + (r & 7) * 2) =
-                __float2bfloat16_rn(pp[h]);
+                __float2bfloat16_rn(pp[0][h]);
           }
         }
-        if (i == d.ntiles - 1 && d.n - i * TM < TM) {
+        if (i == d.ntiles - 1 && d.n - i * C::TT < C::TT) {
           // V rows past the partition's end may hold anything (even NaN); P is 0 there
           // but 0 * NaN is NaN: clear them before the tensor core reads the tile
           const int vs = j % NV;
           failed |= !wait_or_abort(&v_full[vs], (j / NV) & 1, p.err, abort_flag, wl);
-          if (!valid) {
-            uint8_t* v = smem + C::kOffV + vs * kTileBytes + r * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
-              if (!F8) *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
+          for (int u = 0; u < SUB; ++u) {
+            if (!valid[u]) {
+              // e4m3: row u * 128 + r of 128 bytes; bf16: row r in both 64-dim halves
+              uint8_t* v = smem + C::kOffV + vs * kTileBytes + (u * TM + r) * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
+                if (!F8) *reinterpret_cast<uint4*>(v + kRegion + c * 16) = make_uint4(0, 0, 0, 0);
+              }
             }
           }
         }
@@ -1293,7 +1357,7 @@ unsigned long long next_tag() {
 template <int G, bool F8>
 cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t stream) {
   const int bs = a.cache.block_size;
-  const int rows = bs < TM ? bs : TM;
+  const int rows = bs < Cfg<F8>::TT ? bs : Cfg<F8>::TT;  // positions per TMA box
   const uint64_t slots = static_cast<uint64_t>(a.cache.num_blocks) * bs;
   const uint64_t hkv = static_cast<uint64_t>(a.cache.num_kv_heads);
   CUtensorMap tmQ, tmK, tmV, tmSK, tmSV;
