@@ -64,7 +64,8 @@
 //     operand, so one product fills two side-by-side O^T accumulators combined as
 //     O_hi + O_lo / 128 (about 2^-8 relative on P', and an absolute floor near 2^-17,
 //     so small probabilities keep their precision).
-// Per tile that is 4 + 4 MMA instructions (K = 32 bytes each) instead of 20.
+// Per 128 positions that is 4 + 4 MMA instructions (K = 32 bytes each) instead of 20;
+// an e4m3 tile is 256 positions (32 KB, as a bf16 tile of 128).
 // Before a CTA ends, its producer waits for every copy it started and its issuer for
 // every MMA it issued (with the full time limit, even when the roles gave up early),
 // so no asynchronous write outlives the CTA's shared and tensor memory.
