@@ -30,7 +30,9 @@
 //           hundred cycles, so the order matters: value first keeps V slots and P
 //           buffers turning over, and scoring ahead lets the next item's first tile be
 //           ready when the softmax gets there;
-//   warps 0-3  softmax: thread r owns position r of a tile (TMEM lane r): per-head
+//   warps 0-3  softmax (and 11-14 for e4m3 with up to 8 heads per kv head, taking the
+//           second 128-position half of each tile): thread r owns position r of its
+//           128 positions of a tile (TMEM lane r): per-head
 //           tile max across the 128 positions, exp2 against a per-item reference max,
 //           P^T to shared memory. O^T is rescaled in TMEM only when a tile's max
 //           exceeds the reference by more than 2^8 (so probabilities stay <= 256,
@@ -134,8 +136,8 @@ struct Cfg {
   static constexpr int kOffV = kOffK + NK * kTileBytes;
   static constexpr int kOffQ = kOffV + NV * kTileBytes;
   static constexpr int kOffP = kOffQ + QN * kQBytes;
-  static constexpr int kOffRed = kOffP + NP * kPBytes;  // [3][4 warps][NQ] + [2][4] floats
-  static constexpr int kRedFloats = 3 * 4 * NQ + 2 * 4;
+  static constexpr int kOffRed = kOffP + NP * kPBytes;  // [3][8 warps][NQ] + [2][8] floats
+  static constexpr int kRedFloats = 3 * 8 * NQ + 2 * 8;  // up to 8 softmax warps
   static constexpr int kOffQs = align_up(kOffRed + kRedFloats * 4, 16);  // [QN][NQ] q scales
   static constexpr int kOffIds = align_up(kOffQs + QN * NQ * 4, 16);
   static constexpr int kOffSched = align_up(kOffIds + QS * kMaxIds * 4, 16);  // [QS] descriptors
@@ -358,14 +360,25 @@ __device__ __forceinline__ void split_e4m3x2(float a, float b, float lo_scale, u
   lo = e4m3x2((a - h.x) * lo_scale, (b - h.y) * lo_scale, unused);
 }
 
+// Softmax groups: for e4m3 with up to 8 heads per kv head, two groups of four warps take
+// the two 128-position halves of a tile side by side (one position per thread, 480
+// threads, 128 registers each); otherwise one group takes the whole tile.
 template <int G, bool F8>
-__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
+constexpr int kSoftGroups = (F8 && G <= 8) ? 2 : 1;
+template <int G, bool F8>
+constexpr int kThreadsOf = kSoftGroups<G, F8> == 2 ? 480 : kThreads;
+
+template <int G, bool F8>
+__global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmSK,
     const __grid_constant__ CUtensorMap tmSV, const TcParams p) {
   static_assert(G >= 1 && G <= NQ, "query heads per kv head");
   using C = Cfg<F8>;
   constexpr int NK = C::NK, NV = C::NV, NSC = C::NSC;
+  constexpr int SG = kSoftGroups<G, F8>;
+  constexpr int kSoftThreads = 128 * SG;
+  static_assert(SG == 1 || C::kSub == SG, "two softmax groups take one half of a tile each");
   constexpr int kRegion = C::kRegion, kTileBytes = C::kTileBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -429,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     }
     for (int i = 0; F8 && i < NSC; ++i) {
       mbar_init(&ksc_full[i], 1);
-      mbar_init(&ksc_empty[i], 4);
+      mbar_init(&ksc_empty[i], 4 * SG);
     }
     for (int i = 0; F8 && i < QN; ++i) mbar_init(&q_ready[i], 1);
     for (int i = 0; i < QN; ++i) {
@@ -438,10 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], 4 * SG);
     }
     for (int i = 0; i < NP; ++i) {
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 4 * SG);
       mbar_init(&pv_done[i], 1);
     }
     for (int i = 0; i < NO; ++i) {
@@ -920,20 +933,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       tc_commit(mma_drain);
       mbar_wait(mma_drain, 0, p.err);
     }
-  } else if (warp < 4) {
-    // ======================================================== softmax warps 0-3
-    // Control flow stays uniform across the 128 threads: a wait that fails (time
+  } else if (warp < 4 || (SG == 2 && warp >= 11)) {
+    // ======================================================== softmax warps 0-3 (+ 11-14)
+    // Control flow stays uniform across the softmax threads: a wait that fails (time
     // limit, or another role gave up) only marks `failed`; the group leaves together
     // at an item boundary through a barrier vote, so no thread can strand the others
     // at a named barrier.
-    const int r = tid;  // position within a tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int sg = warp < 4 ? 0 : 1;         // softmax group
+    const int quad = warp & 3;               // TMEM lane quadrant of this warp
+    const int wi = sg * 4 + quad;            // this warp's slot in the exchange buffers
+    const int r = quad * 32 + lane;          // position within a 128-position product = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    // the tile's 128-position products this thread takes: its group's half with two
+    // groups, else every one
+    constexpr int PT = SG == 2 ? 1 : C::kSub;
+    auto sub_of = [&](int t) { return SG == 2 ? sg : t; };
     // e4m3: byte offsets of this thread's positions' scales within a tile's scale area
-    int soff[C::kSub];
+    int soff[PT];
 #pragma unroll
-    for (int u = 0; u < C::kSub; ++u) {
-      const int pos = u * TM + r;
-      soff[u] = (pos / srows) * sstride + (pos % srows) * 4;
+    for (int t = 0; t < PT; ++t) {
+      const int pos = sub_of(t) * TM + r;
+      soff[t] = (pos / srows) * sstride + (pos % srows) * 4;
     }
     int k = 0;
     unsigned j = 0;  // tiles of this CTA done
@@ -947,7 +967,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       float qsg[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) qsg[h] = F8 ? qscale[slot * NQ + h] : 1.f;
-      if (bar_or(1, 128, failed)) break;  // every thread has read the descriptor
+      if (bar_or(1, kSoftThreads, failed)) break;  // every thread has read the descriptor
       if (tid == 0) mbar_arrive(&item_empty[slot]);
       if (d.stop) {
         if (tid == 0) {  // tell the epilogue warps, once they have read slot k % NO
@@ -968,14 +988,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         lp[h] = 0.f;
         R[h] = -INFINITY;  // e4m3: O's reference, unset until a tile has a non-zero V scale
       }
-      // A tile is SUB products of 128 positions: thread r owns position r of each
-      // (r and 128 + r for e4m3 tiles of 256).
-      constexpr int SUB = C::kSub;
+      // A tile is kSub products of 128 positions: thread r owns position r of the ones
+      // it takes (see sub_of)
+      constexpr int SUB = PT;
       for (int i = 0; i < d.ntiles; ++i, ++j) {
         const int sb = j % NS;
         bool valid[SUB];
 #pragma unroll
-        for (int u = 0; u < SUB; ++u) valid[u] = i * C::TT + u * TM + r < d.n;
+        for (int u = 0; u < SUB; ++u) valid[u] = i * C::TT + sub_of(u) * TM + r < d.n;
         // e4m3: the tile's K and V row scales first: they land with the tiles, well
         // before the score MMA is done, so their waits and reads overlap it
         float skr[SUB], svr[SUB];  // svr: this position's V scale (0 past the partition)
@@ -1005,7 +1025,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         float sv[SUB][G];
 #pragma unroll
         for (int u = 0; u < SUB; ++u) {
-          const uint32_t ts = tmem + sb * C::kSCols + u * NQ * kQTerms + lane_off;
+          const uint32_t ts = tmem + sb * C::kSCols + sub_of(u) * NQ * kQTerms + lane_off;
           tmem_ld_cols<G>(ts, sv[u]);
           if constexpr (F8) {
             // S = products with the hi, mid and lo q terms, summed
@@ -1034,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           }
         }
         // per-head max over the tile: warp shuffles, then across the 4 warps
-        float* rb = red + (j & 1) * 4 * NQ;
+        float* rb = red + (j & 1) * 8 * NQ;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float v = x[0][h];
@@ -1042,30 +1062,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           for (int u = 1; u < SUB; ++u) v = fmaxf(v, x[u][h]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) rb[warp * NQ + h] = v;
+          if (lane == 0) rb[wi * NQ + h] = v;
         }
-        float* svb = red + 3 * 4 * NQ + (j & 1) * 4;  // e4m3: the tile's largest V scale
+        float* svb = red + 3 * 8 * NQ + (j & 1) * 8;  // e4m3: the tile's largest V scale
         if (F8) {
           float v = svr[0];
 #pragma unroll
           for (int u = 1; u < SUB; ++u) v = fmaxf(v, svr[u]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) svb[warp] = v;
+          if (lane == 0) svb[wi] = v;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kSoftThreads);
         bool rescale = false;
+        auto tile_max = [&](int h) {
+          float v = rb[h];
+#pragma unroll
+          for (int w = 1; w < 4 * SG; ++w) v = fmaxf(v, rb[w * NQ + h]);
+          return v;
+        };
         float alpha[G];
         float pp[SUB][G];  // P' (e4m3) or P (bf16) of this thread's positions per head
         if constexpr (F8) {
           // bound of P' over the tile: 2^(max x + log2 max s_v - R)
-          const float lsm = lg2_approx(fmaxf(fmaxf(svb[0], svb[1]), fmaxf(svb[2], svb[3])));
+          float smax = svb[0];
+#pragma unroll
+          for (int w = 1; w < 4 * SG; ++w) smax = fmaxf(smax, svb[w]);
+          const float lsm = lg2_approx(smax);
           float lsv[SUB];
 #pragma unroll
           for (int u = 0; u < SUB; ++u) lsv[u] = lg2_approx(svr[u]);  // -inf for s_v = 0
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
+            const float mx = tile_max(h);
             // l's reference (the row sum stays fp32, only its range matters)
             if (i == 0) {
               m[h] = mx;
@@ -1094,7 +1123,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         } else {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float mx = fmaxf(fmaxf(rb[h], rb[NQ + h]), fmaxf(rb[2 * NQ + h], rb[3 * NQ + h]));
+            const float mx = tile_max(h);
             alpha[h] = 1.f;
             if (i == 0) {
               m[h] = mx;  // reference max of this item (every tile has a valid position)
@@ -1121,7 +1150,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           // swizzle): byte r of chunk u; the lo terms kQRegion after the hi ones
 #pragma unroll
           for (int u = 0; u < SUB; ++u) {
-            uint8_t* pt = smem + C::kOffP + pb * C::kPBytes + u * kPChunk;
+            uint8_t* pt = smem + C::kOffP + pb * C::kPBytes + sub_of(u) * kPChunk;
 #pragma unroll
             for (int h = 0; h < G; h += 2) {
               uint32_t hi, lo;
@@ -1153,7 +1182,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
           for (int u = 0; u < SUB; ++u) {
             if (!valid[u]) {
               // e4m3: row u * 128 + r of 128 bytes; bf16: row r in both 64-dim halves
-              uint8_t* v = smem + C::kOffV + vs * kTileBytes + (u * TM + r) * 128;
+              uint8_t* v = smem + C::kOffV + vs * kTileBytes + (sub_of(u) * TM + r) * 128;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
                 *reinterpret_cast<uint4*>(v + c * 16) = make_uint4(0, 0, 0, 0);
@@ -1162,7 +1191,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
             }
           }
         }
-        if (rescale) {  // uniform across the group: every thread saw the same tile max
+        // uniform across the groups (every thread saw the same tile max); group 0's
+        // warps cover all 128 TMEM lanes of O, so it rescales alone
+        if (sg == 0 && rescale) {
           // O holds the value MMAs up to tile j-1: wait for the last of them
           const unsigned t = j - 1;
           failed |= !wait_or_abort(&pv_done[t % NP], (t / NP) & 1, p.err, abort_flag, wl);
@@ -1190,15 +1221,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       // hand the item to the epilogue warps: l per head (the per-position shares summed
       // over the 128 threads), the reference max and, for e4m3, O's factor 2^(R - m);
       // O^T stays in TMEM
-      float* lb = red + 2 * 4 * NQ;
+      float* lb = red + 2 * 8 * NQ;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float v = lp[h];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) lb[warp * NQ + h] = v;
+        if (lane == 0) lb[wi * NQ + h] = v;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kSoftThreads);
       if (tid == 0) {
         const int b = k % NO;
         if (k >= NO)
@@ -1210,13 +1241,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             em[h] = m[h];
-            em[NQ + h] = lb[h] + lb[NQ + h] + lb[2 * NQ + h] + lb[3 * NQ + h];
+            float L = 0.f;
+            for (int w = 0; w < 4 * SG; ++w) L += lb[w * NQ + h];
+            em[NQ + h] = L;
             em[2 * NQ + h] = (F8 && R[h] > -INFINITY) ? ex2_approx(R[h] - m[h]) : (F8 ? 0.f : 1.f);
           }
           mbar_arrive(&epi_full[b]);
         }
       }
-      if (bar_or(1, 128, failed)) break;
+      if (bar_or(1, kSoftThreads, failed)) break;
       ++k;
     }
   } else if (warp < 10) {
@@ -1390,7 +1423,8 @@ cudaError_t launch_tc_t(const DecodeLaunch& a, const TcParams& p, cudaStream_t s
   int grid = sm_count();
   if (static_cast<unsigned>(grid) > p.total_items) grid = static_cast<int>(p.total_items);
   if (grid < 1) grid = 1;
-  decode_tc_kernel<G, F8><<<grid, kThreads, smem_bytes, stream>>>(tmQ, tmK, tmV, tmSK, tmSV, p);
+  decode_tc_kernel<G, F8><<<grid, kThreadsOf<G, F8>, smem_bytes, stream>>>(tmQ, tmK, tmV, tmSK,
+                                                                          tmSV, p);
   return cudaGetLastError();
 }
 
