@@ -571,6 +571,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
       // The whole warp runs the tile loop (waits and coordinates warp-uniform); one
       // elected lane issues each load. A lane-0 branch with broadcast verdicts cost this
       // warp ~2000 cycles a tile, more than an e4m3 tile's share of the DRAM time.
+#pragma unroll 1
       for (int i = 0; i < ntiles; ++i) {
         // K of tile jk: its slot frees when the score MMA of tile jk - NK is done
         const int ks = jk % NK;
@@ -588,6 +589,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
           uint8_t* kdst = smem + C::kOffK + ks * kTileBytes;
           mbar_arrive_expect_tx_w(&k_full[ks], kTileBytes);
           if (F8) mbar_arrive_expect_tx_w(&ksc_full[kl], C::TT * 4);
+#pragma unroll 1
           for (int b = 0; b < nbox; ++b) {
             const int row = row_of(idc, first_blk, t0 + i * C::TT + b * rows);
             if (F8) {
@@ -611,6 +613,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
           uint8_t* vdst = smem + C::kOffV + vs * kTileBytes;
           mbar_arrive_expect_tx_w(&v_full[vs], kTileBytes);
           if (F8) mbar_arrive_expect_tx_w(&vsc_full[vs], C::TT * 4);
+#pragma unroll 1
           for (int b = 0; b < nbox; ++b) {
             const int row = row_of(idc, first_blk, t0 + i * C::TT + b * rows);
             if (F8) {
@@ -635,18 +638,23 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
     // waiting for the last phase of each slot is enough; on the normal path these
     // completed long ago. Full time limit: these copies always complete.
     if (lane == 0) {
+#pragma unroll 1
       for (unsigned t = jk > static_cast<unsigned>(NK) ? jk - NK : 0; t < jk; ++t)
         mbar_wait(&k_full[t % NK], (t / NK) & 1, p.err);
+#pragma unroll 1
       for (unsigned t = jv > static_cast<unsigned>(NV) ? jv - NV : 0; t < jv; ++t)
         mbar_wait(&v_full[t % NV], (t / NV) & 1, p.err);
       if (F8) {
+#pragma unroll 1
         for (unsigned t = jk > static_cast<unsigned>(NSC) ? jk - NSC : 0; t < jk; ++t)
           mbar_wait(&ksc_full[t % NSC], (t / NSC) & 1, p.err);
+#pragma unroll 1
         for (unsigned t = jv > static_cast<unsigned>(NV) ? jv - NV : 0; t < jv; ++t)
           mbar_wait(&vsc_full[t % NV], (t / NV) & 1, p.err);
       } else {
         // a q load whose slot took a later item has landed (the slot was handed on only
         // after the issuer had waited for it); only the others are waited for here
+#pragma unroll 1
         for (int t = kq > QN ? kq - QN : 0; t < kq; ++t)
           if (t + QN >= npub) mbar_wait(&item_full[t % QN], (t / QN) & 1, p.err);
       }
@@ -694,6 +702,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
         const int t0 = p.shared_len + part * p.partition_size;
         if (t0 >= ctx) {
           if (part == 0 && p.shared_len == 0) {  // empty context: a zero output row
+#pragma unroll 1
             for (int i = lane; i < G * HD; i += 32)
               p.out[(static_cast<int64_t>(s) * Hq + g * G) * HD + i] = __float2bfloat16(0.f);
             // and no last position to store a new row at
@@ -707,6 +716,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
         first_blk = t0 >> p.bs_log2;
         const int nb = ((t0 + ntiles * C::TT - 1) >> p.bs_log2) - first_blk + 1;
         int* idb = ids + slot * kMaxIds;
+#pragma unroll 1
         for (int i = lane; i < nb && i < kMaxIds; i += 32) {
           const int b = first_blk + i;
           int id = b < p.max_blocks
@@ -1330,6 +1340,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
             const int64_t base = (row0 + h) * p.max_parts;
             const int np = d.nparts;
             float M = -INFINITY;
+#pragma unroll 1
             for (int q0 = 0; q0 < np; q0 += CH) {
               float mm[CH];
 #pragma unroll
@@ -1339,6 +1350,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
               for (int i = 0; i < CH; ++i) M = fmaxf(M, mm[i]);
             }
             float Ls = 0.f, acc = 0.f;
+#pragma unroll 1
             for (int q0 = 0; q0 < np; q0 += CH) {
               float2 ml[CH];
               float oo[CH];

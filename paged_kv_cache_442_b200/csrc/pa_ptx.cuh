@@ -77,8 +77,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, unsigned parity) {
 
 // Wait until the phase with the given parity has completed. Returns false (and
 // flags a timeout) if it did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, unsigned parity, unsigned* err) {
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -88,13 +87,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
     }
   }
 }
-
-// Bounded wait that also gives up when another role of the CTA already gave up (the
-// roles share `abort_flag`): false on a timeout (flagged, and the flag set) or an abort.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
-                                              volatile int* abort_flag,
-                                              unsigned long long limit_ns) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* err) {
   if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, err);
+}
+
+static __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, unsigned parity, unsigned* err,
+                                                       volatile int* abort_flag,
+                                                       unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -105,6 +105,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, un
       return false;
     }
   }
+}
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, unsigned* err,
+                                              volatile int* abort_flag,
+                                              unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_or_abort_slow(bar, parity, err, abort_flag, limit_ns);
 }
 
 // The same wait run by all 32 lanes of a converged warp, with one answer for the warp
