@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
         tma_load_3d_hint(dst + kRegion, nmap, bar, 64, g, row, keep);
         return;
       }
+#pragma unroll 1
       for (int c = 0; c < nbox; ++c) {
         const int row = block_row(j * BN + c * rows);
         tma_load_3d_hint(dst + c * rows * 128, map, bar, 0, g, row, keep);
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
                                uint64_t* bar) -> bool {
       if (lane == 0) {
         mbar_arrive_expect_tx(patch, kTileBytes);
+#pragma unroll 1
         for (int c = 0; c < nbox; ++c) {
           const int row = block_row(jst * BN + c * rows);
           tma_load_3d(dst + c * rows * 128, map, patch, 0, g, row);
@@ -254,6 +256,7 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
       // row r >= r0 of the tile is new row r - r0 of the sequence: 16 vectors each
       const int r0 = first - jst * BN;
       const int nr = min(BN - r0, n_new);
+#pragma unroll 1
       for (int i = lane; i < nr * 16; i += 32) {
         const int r = r0 + (i >> 4), c = i & 15;  // 16-byte chunk c holds dims 8c..8c+7
         const uint4 v =
@@ -280,6 +283,7 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
       }
     }
     int k_issued = 0, v_issued = 0;
+#pragma unroll 1
     for (int j = 0; j < nmax; ++j) {
       const int ks = j % NK;
       if (j >= NK && !wwait(&k_empty[ks], ((j / NK) - 1) & 1)) break;
@@ -303,8 +307,10 @@ __global__ void __launch_bounds__(kStore ? 352 : 320, 1) prefill_kernel(
     // so waiting for those is enough; on the normal path they completed long ago.
     if (lane == 0) {
       mbar_wait(bar_q, 0, p.err);
+#pragma unroll 1
       for (int t = k_issued - NK > 0 ? k_issued - NK : 0; t < k_issued; ++t)
         mbar_wait(&k_full[t % NK], (t / NK) & 1, p.err);
+#pragma unroll 1
       for (int t = v_issued - NV > 0 ? v_issued - NV : 0; t < v_issued; ++t)
         mbar_wait(&v_full[t % NV], (t / NV) & 1, p.err);
       // a straddling tile's pool copy whose wait gave up may still be in flight

@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     const uint64_t keep = policy_evict_last();  // the prefix is read by every CTA of g
     auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
       mbar_arrive_expect_tx(bar, kTileBytes);
+#pragma unroll 1
       for (int c = 0; c < nbox; ++c) {
         const int pos = j * BN + c * rows;
         int id = __ldg(p.shared_blocks + (pos >> p.bs_log2));
@@ -176,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
       }
     }
     int k_issued = 0, v_issued = 0;
+#pragma unroll 1
     for (int j = 0; j < ntiles; ++j) {
       const int ks = j % NK;
       if (j >= NK && !wwait(&k_empty[ks], ((j / NK) - 1) & 1)) break;
@@ -188,8 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     }
     if (lane == 0) {
       mbar_wait(bar_q, 0, p.err);
+#pragma unroll 1
       for (int t = k_issued - NK > 0 ? k_issued - NK : 0; t < k_issued; ++t)
         mbar_wait(&k_full[t % NK], (t / NK) & 1, p.err);
+#pragma unroll 1
       for (int t = v_issued - NV > 0 ? v_issued - NV : 0; t < v_issued; ++t)
         mbar_wait(&v_full[t % NV], (t / NV) & 1, p.err);
     }
@@ -233,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
         return true;
       };
       bool ok = warp_wait_or_abort(bar_q, 0, p.err, abort_flag, p.wait_ns);
+#pragma unroll 1
       for (int u = 0; ok && u < nu; ++u) ok = score(u, 0);
+#pragma unroll 1
       for (int j = 0; ok && j < ntiles; ++j) {
         for (int u = 0; ok && u < nu; ++u) {
           ok = pv(u, j);
@@ -251,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     // would hold up the producer's first loads by tens of microseconds.)
     {
       const int nsb = p.shared_len >> p.bs_log2;
+#pragma unroll 1
       for (int i = tid; i < p.units * spt * nsb; i += 8 * 32) {
         const int s = s0 + i / nsb, b = i % nsb;
         if (s >= p.num_seqs || (b << p.bs_log2) >= __ldg(p.context_lens + s)) continue;
@@ -274,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) shared_prefix_kernel(
     const int vis = ctx < p.shared_len ? (ctx > 0 ? ctx : 0) : p.shared_len;
     float m = -INFINITY, l = 0.f;
     bool failed = false;
+#pragma unroll 1
     for (int j = 0; j < ntiles; ++j) {
       failed |= !wait_or_abort(&s_full[u], j & 1, p.err, abort_flag, p.wait_ns);
       tc_fence_after();
