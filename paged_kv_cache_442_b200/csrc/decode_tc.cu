@@ -426,6 +426,33 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
   const int srows = bs < C::TT ? bs : C::TT;
   const int sstride = srows * 4 < 128 ? 128 : srows * 4;
 
+  // The scheduler's first item is the CTA's own index: its context length, block ids
+  // and (e4m3) q are read here, before the set-up barrier, so that their latency
+  // overlaps the set-up instead of delaying the first tile
+  constexpr int kPreIds = (kMaxIds + 31) / 32;
+  int pre_ctx = 0;
+  int pre_id[kPreIds];
+  uint2 pre_q[F8 ? G : 1];
+  if (warp == 10 && blockIdx.x < p.total_items) {
+    const int s = (blockIdx.x / p.num_kv_heads) % p.num_seqs;
+    const int part = (blockIdx.x / p.num_kv_heads) / p.num_seqs;
+    pre_ctx = __ldg(p.context_lens + s);
+    const int fb = (p.shared_len + part * p.partition_size) >> p.bs_log2;
+#pragma unroll
+    for (int k = 0; k < kPreIds; ++k) {
+      const int b = fb + lane + 32 * k;
+      pre_id[k] = (lane + 32 * k < kMaxIds && b < p.max_blocks)
+                      ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b)
+                      : -1;
+    }
+    if constexpr (F8) {
+      const uint2* src = reinterpret_cast<const uint2*>(
+          p.q + (static_cast<int64_t>(s) * Hq + (blockIdx.x % p.num_kv_heads) * G) * HD);
+#pragma unroll
+      for (int h = 0; h < G; ++h) pre_q[h] = __ldg(src + h * (HD / 4) + lane);
+    }
+  }
+
   // zero the Q slots and P^T buffers: rows >= G are never written and stay zero
   for (int i = tid; i < (QN * C::kQBytes + NP * C::kPBytes) / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + C::kOffQ)[i] = make_uint4(0, 0, 0, 0);
@@ -673,9 +700,11 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
       if (q >= QS && !wwait(&sched_empty[slot], ((q / QS) - 1) & 1)) break;
       ItemDesc d;
       int first_blk = 0;
+      bool used_pre = false;  // this item's inputs were read before the set-up barrier
       while (true) {
         unsigned idx = 0;
         bool ok = true;
+        const bool pre = first_take;
         if (first_take) {
           idx = blockIdx.x;
           first_take = false;
@@ -694,7 +723,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
         const unsigned rr = idx / p.num_kv_heads;
         const int s = rr % p.num_seqs;
         const int part = rr / p.num_seqs;
-        int ctx = __ldg(p.context_lens + s);
+        int ctx = pre ? pre_ctx : __ldg(p.context_lens + s);
         if (ctx > p.max_context_len) {
           if (lane == 0 && part == 0) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
           ctx = p.max_context_len;
@@ -716,18 +745,27 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
         first_blk = t0 >> p.bs_log2;
         const int nb = ((t0 + ntiles * C::TT - 1) >> p.bs_log2) - first_blk + 1;
         int* idb = ids + slot * kMaxIds;
-#pragma unroll 1
-        for (int i = lane; i < nb && i < kMaxIds; i += 32) {
-          const int b = first_blk + i;
-          int id = b < p.max_blocks
-                       ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b)
-                       : -1;
+        auto put_id = [&](int i, int id) {
           if (id < 0 || id >= p.num_blocks) {
-            if ((b << p.bs_log2) < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
+            if (((first_blk + i) << p.bs_log2) < ctx) flag_error(p.err, PA_DEV_ERR_BAD_INDEX);
             id = 0;  // in-bounds stand-in; positions past ctx are masked
           }
           idb[i] = id;
+        };
+        if (pre) {
+#pragma unroll
+          for (int k = 0; k < kPreIds; ++k)
+            if (lane + 32 * k < nb && lane + 32 * k < kMaxIds) put_id(lane + 32 * k, pre_id[k]);
+        } else {
+#pragma unroll 1
+          for (int i = lane; i < nb && i < kMaxIds; i += 32) {
+            const int b = first_blk + i;
+            put_id(i, b < p.max_blocks
+                          ? __ldg(p.block_tables + static_cast<int64_t>(s) * p.max_blocks + b)
+                          : -1);
+          }
         }
+        used_pre = pre;
         const int shared = p.shared_len > 0 ? 1 : 0;
         d.s = s; d.g = g; d.p = part + shared; d.t0 = t0; d.n = n; d.ntiles = ntiles;
         d.nparts = shared + (ctx - p.shared_len + p.partition_size - 1) / p.partition_size;
@@ -754,7 +792,7 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
             p.q + (static_cast<int64_t>(d.s) * Hq + d.g * G) * HD);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const uint2 raw = __ldg(src + h * (HD / 4) + lane);
+          const uint2 raw = used_pre ? pre_q[h] : __ldg(src + h * (HD / 4) + lane);
           const float f0 = bf16lo_to_f32(raw.x), f1 = bf16hi_to_f32(raw.x);
           const float f2 = bf16lo_to_f32(raw.y), f3 = bf16hi_to_f32(raw.y);
           float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
