@@ -1369,25 +1369,18 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
         }
         named_bar_sync(2, 128);
         if (*last_flag) {
-          // this CTA completed the last partition of (s, g): merge all of them. The
-          // partials are read eight partitions at a time with independent loads (one
-          // round trip per chunk, not one per partition)
+          // this CTA completed the last partition of (s, g): merge all of them. Each
+          // head's partials are read eight partitions at a time in one pass (m, l and
+          // this thread's o element together, an online max across the chunks), and no
+          // output is stored before every head's loads, so the loads of all heads can be
+          // in flight together: one round trip per chunk, not two per head and chunk
           constexpr int CH = 8;
+          float res[G];
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const int64_t base = (row0 + h) * p.max_parts;
             const int np = d.nparts;
-            float M = -INFINITY;
-#pragma unroll 1
-            for (int q0 = 0; q0 < np; q0 += CH) {
-              float mm[CH];
-#pragma unroll
-              for (int i = 0; i < CH; ++i)
-                mm[i] = q0 + i < np ? __ldcg(p.ws_ml + (base + q0 + i) * 2) : -INFINITY;
-#pragma unroll
-              for (int i = 0; i < CH; ++i) M = fmaxf(M, mm[i]);
-            }
-            float Ls = 0.f, acc = 0.f;
+            float M = -INFINITY, Ls = 0.f, acc = 0.f;
 #pragma unroll 1
             for (int q0 = 0; q0 < np; q0 += CH) {
               float2 ml[CH];
@@ -1399,15 +1392,25 @@ __global__ void __launch_bounds__(kThreadsOf<G, F8>, 1) decode_tc_kernel(
                            : make_float2(-INFINITY, 0.f);
                 oo[i] = in ? __ldcg(p.ws_o + (base + q0 + i) * HD + dl) : 0.f;
               }
+              float Mc = M;
+#pragma unroll
+              for (int i = 0; i < CH; ++i) Mc = fmaxf(Mc, ml[i].x);
+              // every partition has a finite max (it holds at least one position)
+              const float r = ex2_approx(M - Mc);  // 0 on the first chunk (M = -inf)
+              Ls *= r;
+              acc *= r;
 #pragma unroll
               for (int i = 0; i < CH; ++i) {
-                const float f = ex2_approx(ml[i].x - M);
+                const float f = ex2_approx(ml[i].x - Mc);
                 Ls += ml[i].y * f;
                 acc += oo[i] * f;
               }
+              M = Mc;
             }
-            p.out[(row0 + h) * HD + dl] = __float2bfloat16_rn(acc / Ls);
+            res[h] = acc / Ls;
           }
+#pragma unroll
+          for (int h = 0; h < G; ++h) p.out[(row0 + h) * HD + dl] = __float2bfloat16_rn(res[h]);
         }
       }
       if (bar_or(2, 128, failed)) break;  // also orders last_flag's reuse
